@@ -1,0 +1,474 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused gated-MLP hot path on B200.
+
+One step = the whole MLP block (RMSNorm -> interleaved gate-up -> SiLU*up ->
+down projection) over one batch of token rows for every layer of the
+workload, through the library's C ABI.  Default workload: a Phi-3-mini-shaped
+decode layer (M=1, d=3072, I=8192, bf16) over 32 independent layers' weights,
+4.8 GB of weights per GPU, far beyond the 126 MB L2, so no L2 flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...     # the fp64 CPU oracle, timed alone
+
+Multi-GPU: launched by torch.distributed.run, one rank per GPU; the path has
+no exchange step, so every rank runs its own replica of the workload (weak
+scaling) and the reported time is the max over ranks.
+
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+EPS = 1e-5
+TILE_T = 16
+METRIC = "fused-MLP weight-stream GB/s (% B200 HBM peak) and tokens/s per layer at 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def algorithmic_bytes(M: int, d: int, I: int, residual: bool = False) -> int:
+    """Bytes the MLP block must move once: weights 6dI, x 2Md, gamma 2d, out 4Md (+ residual 2Md)."""
+    return 6 * d * I + 2 * M * d + 2 * d + 4 * M * d + (2 * M * d if residual else 0)
+
+
+def gateup_bytes(M: int, d: int, I: int) -> int:
+    """Algorithmic bytes of the gate-up kernel: packed weights 4dI, x, gamma, a written 2MI."""
+    return 4 * d * I + 2 * M * d + 2 * d + 2 * M * I
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "token_phase_swiglu_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel, {}).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the GPU works."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self._nvml = pynvml
+            self._handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 -- clocks are reported as unavailable
+            self.error = repr(e)
+            self._handle = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        if self._handle is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        names = sorted(n for n, bit in self.REASONS.items() if self.reasons & bit)
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------
+# the fp64 oracle as a CPU baseline (a bounded sample of the workload)
+# ----------------------------------------------------------------------------
+
+def layer_bits(w: wl.Workload, seed: int, layer: int) -> dict:
+    act = wl.make_activations(w.M, w.d, seed=seed)
+    wts = wl.make_weights(w.d, w.I, w.sigma, seed=seed + layer)
+    return {k: wl.bf16_bits(v) for k, v in {**act, **wts}.items()}
+
+
+def oracle_call(w: wl.Workload, b: dict, ic: int):
+    """One oracle evaluation of the MLP block on an I-slice of `ic` columns.
+
+    Gate/up/down columns are independent terms of Eq(1), so a slice of the
+    intermediate dimension is a proportional share of the layer's work.
+    Returns (algorithmic bytes, seconds).
+    """
+    import oracle
+    wg, wu = b["W_gate"][:ic], b["W_up"][:ic]
+    wd = np.ascontiguousarray(b["W_down"][:, :ic])
+    t0 = time.perf_counter()
+    oracle.fused_mlp_bf16(b["x"], b["gamma"], EPS, wg, wu, wd)
+    return algorithmic_bytes(w.M, w.d, ic), time.perf_counter() - t0
+
+
+def oracle_sample(w: wl.Workload, seconds: float, seed: int = 0):
+    """The oracle on whole layers of the workload for about `seconds` of CPU time."""
+    done, t_total, calls = 0, 0.0, 0
+    while True:
+        b = layer_bits(w, seed, calls % w.layers)
+        nb, dt = oracle_call(w, b, w.I)
+        done += nb
+        t_total += dt
+        calls += 1
+        if t_total >= seconds:
+            break
+    desc = (f"{calls} whole layer(s) of {w.name} (M={w.M}, d={w.d}, I={w.I}) through the fp64 "
+            f"oracle (bf16 decode + numpy), {t_total:.1f} s")
+    return done / t_total / 1e9, desc
+
+
+def run_reference(args) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    b = layer_bits(w, 0, 0)
+    # size one step so that warm-up + timed steps finish within about two minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    _, t_full = oracle_call(w, b, w.I)
+    ic = w.I
+    if t_full > budget:
+        ic = min(w.I, max(8, int(w.I * budget / t_full) // 8 * 8))
+    for _ in range(args.warmup):
+        oracle_call(w, b, ic)
+    t, nbytes = 0.0, 0
+    for _ in range(args.steps):
+        nb, dt = oracle_call(w, b, ic)
+        t += dt
+        nbytes += nb
+    gbs = nbytes / t / 1e9
+    cores = blas_threads()
+    sample = (f"each step: the fp64 oracle (bf16 decode + numpy) on layer 0 of {w.name} "
+              f"(M={w.M}, d={w.d}) restricted to an I-slice of {ic} of {w.I} columns")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w: wl.Workload, args) -> dict:
+    return {"workload": w.name, "M": w.M, "d": w.d, "I": w.I, "layers": w.layers,
+            "tile_T": TILE_T, "dtype_in": "bf16", "out": "f32",
+            "weights_per_gpu_GB": round(w.layers * 6 * w.d * w.I / 1e9, 3),
+            "l2": "no flush: weights streamed per step exceed the 126 MB L2",
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+
+def run_ours(args) -> None:
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import token_phase_swiglu_b200 as fm
+
+    w = wl.WORKLOADS[args.workload]
+    M, d, I, L = w.M, w.d, w.I, w.layers
+    seed0 = 1000 * rank
+
+    # resident weights: packed gate/up and W_down per layer (+ gamma per layer)
+    act = wl.make_activations(M, d, seed=seed0)
+    x = act["x"].to(dev)
+    layers = []
+    for l in range(L):
+        wts = wl.make_weights(d, I, w.sigma, seed=seed0 + l)
+        gamma = wl.normal_bf16(seed0 + l, wl.TID_GAMMA, (d,), mean=1.0, std=0.1).to(dev)
+        wg, wu = wts["W_gate"].to(dev), wts["W_up"].to(dev)
+        packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+        fm.fmlp_pack(wg, wu, TILE_T, packed)
+        torch.cuda.synchronize()
+        del wg, wu
+        layers.append({"packed": packed, "W_down": wts["W_down"].to(dev), "gamma": gamma,
+                       "out": torch.empty(M, d, dtype=torch.float32, device=dev)})
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    a_buf = torch.empty(M, I, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        # the current stream (the capture stream while a graph is being captured)
+        for ly in layers:
+            fm.fmlp_forward(x, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], ly["out"], ws)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up (also the one-time library set-up, before any graph capture)
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            torch.cuda.synchronize()
+            for _ in range(args.warmup):
+                graph.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # noqa: BLE001 -- report and launch from the host instead
+            print(f"bench: CUDA graph capture failed ({e}); launching from the host",
+                  file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+
+    sampler = ClockSampler(dev.index)
+    launches0 = fm.fmlp_kernel_launch_count()
+    with sampler:
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    elapsed_ms = max_over_ranks(e0.elapsed_time(e1))
+    launches = fm.fmlp_kernel_launch_count() - launches0
+    if graph is not None:
+        launches = 2 * L * args.steps   # replays launch the captured kernels: 2 per layer
+    fm_status = fm.fmlp_device_status(ws)
+
+    bytes_step = L * algorithmic_bytes(M, d, I)
+    total_bytes = bytes_step * args.steps * world
+    gbs = total_bytes / (elapsed_ms / 1e3) / 1e9
+    ms_step = elapsed_ms / args.steps
+    tok_per_s_layer = M * L * args.steps * world / (elapsed_ms / 1e3)
+
+    # per-kernel durations: the same step through the two stage calls, each
+    # launch bracketed by events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)]
+    gu_ms, dn_ms = [], []
+    kernel_steps = max(1, min(args.steps, 50))
+    for _ in range(kernel_steps):
+        for ly, (a0, a1, a2) in zip(layers, ev):
+            a0.record(stream)
+            fm.fmlp_gate_up_swiglu(x, ly["gamma"], EPS, ly["packed"], TILE_T, a_buf, ws,
+                                   stream=stream)
+            a1.record(stream)
+            fm.fmlp_down_proj(a_buf, ly["W_down"], ly["out"], ws, stream=stream)
+            a2.record(stream)
+        torch.cuda.synchronize()
+        for a0, a1, a2 in ev:
+            gu_ms.append(a0.elapsed_time(a1))
+            dn_ms.append(a1.elapsed_time(a2))
+    gu_avg = max_over_ranks(statistics.mean(gu_ms))
+    dn_avg = max_over_ranks(statistics.mean(dn_ms))
+
+    # end to end: host x in (pinned), the layers, host outputs back, every step
+    x_host = act["x"].pin_memory()
+    outs_host = torch.empty(L, M, d, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_steps = max(1, min(args.steps, 200))
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        for li, ly in enumerate(layers):
+            fm.fmlp_forward(x_dev, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], ly["out"],
+                            ws, stream=stream)
+        for li, ly in enumerate(layers):
+            outs_host[li].copy_(ly["out"], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_gbs = bytes_step * e2e_steps * world / (e2e_ms / 1e3) / 1e9
+
+    peaks = measured_peaks()
+    if "hbm_gbs" in peaks:
+        peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+    else:
+        peak, peak_src = FALLBACK_HBM_GBS, "fallback"
+    gu_achieved = gateup_bytes(M, d, I) / (gu_avg / 1e3) / 1e9
+    traffic = recorded_traffic("gateup_swiglu_gemv", w.name)
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, desc = oracle_sample(w, args.cpu_seconds, seed=seed0)
+            cpu = {"value": round(v, 4), "unit": "GB/s", "cores": blas_threads(),
+                   "kind": "oracle", "sample": desc}
+        line = {
+            "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w, args),
+            "hbm_frac": round(gbs / world / peak, 4),
+            "tokens_per_s_per_layer": round(tok_per_s_layer, 1),
+            "roofline": {"bound": "hbm", "kernel": "gateup_swiglu_gemv",
+                         "achieved": round(gu_achieved, 2), "peak": peak, "peak_source": peak_src,
+                         "unit": "GB/s", "frac": round(gu_achieved / peak, 4),
+                         "traffic": traffic,
+                         "algorithmic_bytes_per_launch": gateup_bytes(M, d, I),
+                         "avg_launch_ms": round(gu_avg, 5)},
+            "kernels": {"gateup_swiglu_gemv_ms": round(gu_avg, 5),
+                        "down_gemv_ms": round(dn_avg, 5),
+                        "down_gemv_GBps": round((2 * d * I + 2 * M * I + 4 * M * d) /
+                                                (dn_avg / 1e3) / 1e9, 2)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                    "d2h_bytes_per_step": outs_host.numel() * outs_host.element_size()},
+            "gpu_launches": launches,
+            "cuda_graph": graph is not None,
+            "device_status": fm.fmlp_status_string(fm_status),
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="phi3_decode", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--no-graph", action="store_true", help="launch each step from the host")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,155 @@
+/*
+ * fmlp.h -- C ABI of the B200 fused gated-MLP library (libfmlp.so).
+ *
+ * The library computes the MLP block of a decoder-only transformer layer over
+ * a small batch of token rows:
+ *
+ *     r[m] = 1 / sqrt(mean_k x[m,k]^2 + eps)                 RMSNorm
+ *     h    = x * r * gamma
+ *     a    = SiLU(h W_gate^T) * (h W_up^T),  SiLU(t) = t/(1+e^-t)
+ *     out  = a W_down^T  (+ residual)
+ *
+ * Sources: "FastTPS: An Optimized Method for LLM Token Phase for AI
+ * Accelerators" (xllm-io paper review), section 三: Eq(1), the MLP execution
+ * flow (RMSNorm -> interleaved gate-up Matmul -> siLu_Mul -> down projection)
+ * and component 3 "Fusion MLP"; section 五, Fusion MLP Steps 1-3; and
+ * "CUDAカーネル融合で推論が最大10%高速化" (blog.cecily.jp), the llama.cpp PR
+ * #29948 paragraph on alternating gate/up rows.  The pages define no API;
+ * the calls below are this library's own.
+ *
+ * Conventions for every call
+ *   - All tensors are dense, row-major, in DEVICE memory owned by the caller.
+ *     bf16 is IEEE bfloat16 (2 bytes), f32 is IEEE binary32.  Every pointer
+ *     must be 16-byte aligned.  The library never writes an input and never
+ *     allocates device memory per call.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous on it; a returned FMLP_OK means the work was enqueued.
+ *   - Arguments are validated on the host first; on any validation failure
+ *     nothing is launched and FMLP_ERR_INVALID_ARG or FMLP_ERR_UNSUPPORTED is
+ *     returned.  A CUDA launch or runtime failure returns FMLP_ERR_CUDA (the
+ *     CUDA error code is kept for fmlp_last_cuda_error()).  There is no CPU
+ *     fallback: without a usable sm_100 device every compute call fails.
+ *   - Sizes: d (hidden) and I (intermediate) must be positive multiples of 8
+ *     (rows are whole 16-byte vectors), d <= 32768, I <= 131072.  M (token
+ *     rows) may be 0, which is a no-op.
+ */
+#ifndef FMLP_H
+#define FMLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(FMLP_BUILD) && defined(__GNUC__)
+#define FMLP_API __attribute__((visibility("default")))
+#else
+#define FMLP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fmlp_status {
+  FMLP_OK = 0,
+  FMLP_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, bad eps, small workspace */
+  FMLP_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement        */
+  FMLP_ERR_CUDA = 3,         /* a CUDA call or launch failed                             */
+  FMLP_ERR_TIMEOUT = 4       /* a bounded device-side wait expired (device status word)  */
+} fmlp_status;
+
+/*
+ * fmlp_pack -- interleave W_gate and W_up rows into one matrix (step a0).
+ *
+ * FastTPS section 三, component 3 (gate/up projections interleaved into one
+ * large matmul) and the llama.cpp PR paragraph (gate and up rows alternate).
+ * With tile T, packed rows [2T*t, 2T*t+T) are W_gate rows [T*t, T*t+T) and
+ * packed rows [2T*t+T, 2T*(t+1)) are the W_up rows [T*t, T*t+T):
+ *     packed[2T*t + j]     = W_gate[T*t + j]
+ *     packed[2T*t + T + j] = W_up  [T*t + j],   0 <= j < T.
+ * A pure permutation of rows: the bytes are copied unchanged.
+ *
+ *   W_gate, W_up : bf16 [I x d]   (nn.Linear layout: out x in)
+ *   d, I         : d % 8 == 0, I % 8 == 0
+ *   tile_T       : tile_T % 8 == 0 and I % tile_T == 0 (16 is the canonical tile)
+ *   packed       : bf16 [2I x d], caller-allocated, must not overlap the inputs
+ */
+FMLP_API fmlp_status fmlp_pack(const void* W_gate, const void* W_up, int64_t d, int64_t I,
+                      int tile_T, void* packed, void* stream);
+
+/*
+ * fmlp_workspace_bytes -- bytes of device workspace fmlp_forward needs for
+ * (M, d, I).  The workspace holds a device status word, the bf16
+ * intermediate a [M x I] and per-path scratch.  A workspace must be
+ * zero-filled once before its first use; the library leaves its control
+ * words at zero after every call.  Returns 0 for invalid sizes.
+ */
+FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
+
+/*
+ * fmlp_forward -- the whole MLP block (steps a1-a6): RMSNorm, interleaved
+ * gate-up contraction, SiLU*up epilogue, down projection, optional residual.
+ *
+ *   x          : bf16 [M x d] token rows
+ *   M          : token rows, >= 0
+ *   gamma      : bf16 [d] RMSNorm weight (multiplies directly)
+ *   eps        : RMSNorm epsilon, finite and > 0
+ *   packed_Wgu : bf16 [2I x d] from fmlp_pack with the same tile_T
+ *   W_down     : bf16 [d x I]
+ *   residual   : bf16 [M x d] added to the output, or NULL
+ *   out        : f32 [M x d]
+ *   workspace  : >= fmlp_workspace_bytes(M, d, I) bytes, zero-filled before
+ *                first use, not shared by calls that may overlap on the GPU
+ *
+ * Precision: x*gamma is formed exactly in f32 and the contraction keeps it at
+ * f32 precision (CUDA-core path) or as an exact hi+lo bf16 pair (tensor-core
+ * path); accumulation is f32; a is rounded once to bf16 (round to nearest
+ * even); out is f32.
+ */
+FMLP_API fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
+                         const void* packed_Wgu, int tile_T, const void* W_down,
+                         int64_t d, int64_t I, const void* residual, float* out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fmlp_gate_up_swiglu -- steps a1-a4 alone: writes the bf16 intermediate
+ *     a[m,i] = bf16( SiLU(r[m] * g[m,i]) * r[m] * u[m,i] )
+ * with g, u the contractions of x*gamma with the gate and up rows of
+ * packed_Wgu.  Arguments as in fmlp_forward; `a` is bf16 [M x I] and must not
+ * overlap the workspace.
+ */
+FMLP_API fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* gamma, float eps,
+                                const void* packed_Wgu, int tile_T, int64_t d, int64_t I,
+                                void* a, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
+ * fmlp_down_proj -- steps a5-a6 alone: out = a W_down^T (+ residual).
+ *   a : bf16 [M x I]; other arguments as in fmlp_forward.
+ */
+FMLP_API fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t d,
+                           int64_t I, const void* residual, float* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * fmlp_device_status -- synchronise `stream`, read the device status word in
+ * `workspace` and reset it to zero.  Returns FMLP_ERR_TIMEOUT if a kernel
+ * gave up a bounded wait since the last check, FMLP_OK otherwise (or
+ * FMLP_ERR_CUDA / FMLP_ERR_INVALID_ARG).
+ */
+FMLP_API fmlp_status fmlp_device_status(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+FMLP_API const char* fmlp_status_string(fmlp_status status);
+
+/* The cudaError_t behind the calling thread's most recent FMLP_ERR_CUDA (0 if none). */
+FMLP_API int fmlp_last_cuda_error(void);
+
+/* Kernels this library has enqueued in this process so far (all threads, all
+ * devices; a launch captured into a CUDA graph counts once, at capture). */
+FMLP_API uint64_t fmlp_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMLP_H */

@@ -34,6 +34,7 @@ from .fmlp import (  # noqa: F401
     rms_inv,
     rmsnorm,
     silu,
+    swiglu_intermediate,
     gated_mlp,
     fused_mlp,
     interleaved_rows,

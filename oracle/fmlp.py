@@ -98,6 +98,18 @@ def silu(t: np.ndarray) -> np.ndarray:
         return t / (1.0 + np.exp(-t))
 
 
+def swiglu_intermediate(h, W_gate, W_up) -> np.ndarray:
+    """a = SiLU(h W_gate^T) * (h W_up^T) for token rows h [M x d] -> [M x I].
+
+    [FastTPS] Eq(1) inner part and the siLu_Mul step: SiLU on the gate branch,
+    elementwise product with the up branch.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    g = h @ np.asarray(W_gate, dtype=np.float64).T
+    u = h @ np.asarray(W_up, dtype=np.float64).T
+    return silu(g) * u
+
+
 def gated_mlp(h, W_gate, W_up, W_down, intermediate=None) -> np.ndarray:
     """Eq(1) of [FastTPS] for token rows h [M x d]:  O = (SiLU(h Wg^T) * (h Wu^T)) Wd^T.
 
@@ -109,10 +121,7 @@ def gated_mlp(h, W_gate, W_up, W_down, intermediate=None) -> np.ndarray:
     projection -- the precision of the intermediate the fused design stores
     (the bf16 simulation of section 六).  The default keeps a in binary64.
     """
-    h = np.asarray(h, dtype=np.float64)
-    g = h @ np.asarray(W_gate, dtype=np.float64).T
-    u = h @ np.asarray(W_up, dtype=np.float64).T
-    a = silu(g) * u
+    a = swiglu_intermediate(h, W_gate, W_up)
     if intermediate == "bf16":
         a = round_to_bf16(a)
     elif intermediate is not None:

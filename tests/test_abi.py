@@ -1,0 +1,119 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects invalid arguments on the host before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import token_phase_swiglu_b200 as fm
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "fmlp.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"FMLP_API\s+[\w\s\*]+?\b(fmlp_\w+)\s*\(", src)
+
+
+def test_header_declares_the_binding_surface():
+    names = declared_functions()
+    assert len(names) == len(set(names))
+    assert set(names) == set(fm.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fm.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_exports_nothing_else_from_the_library():
+    # -fvisibility=hidden keeps internal kernels/launchers out of the dynamic table
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", fm.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    ours = {ln.split()[-1] for ln in out.splitlines() if " T " in ln and "fmlp" in ln}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings():
+    for s in range(5):
+        assert fm.fmlp_status_string(s).startswith("FMLP_")
+    assert "unknown" in fm.fmlp_status_string(99)
+
+
+def test_workspace_bytes():
+    L = fm.lib
+    assert L.fmlp_workspace_bytes(4, 256, 688) >= 256 + 4 * 688 * 2
+    assert L.fmlp_workspace_bytes(0, 256, 688) >= 256
+    assert L.fmlp_workspace_bytes(128, 8192, 28672) >= 128 * 28672 * 2
+    # invalid sizes give 0
+    assert L.fmlp_workspace_bytes(1, 255, 688) == 0
+    assert L.fmlp_workspace_bytes(1, 256, 690) == 0
+    assert L.fmlp_workspace_bytes(-1, 256, 688) == 0
+    assert L.fmlp_workspace_bytes(1, 65536, 688) == 0
+    for M in (1, 7, 2048):
+        assert L.fmlp_workspace_bytes(M, 4096, 14336) % 256 == 0
+
+
+# Fake, 16-byte aligned addresses: every call below fails validation and returns
+# before touching the device, so nothing is dereferenced.
+A = 0x10000
+B = 0x20000
+MIS = 0x30008
+
+
+def _fwd(**kw):
+    args = dict(x=A, M=4, gamma=A, eps=1e-5, P=A, T=16, Wd=A, d=256, I=688, res=None, out=B,
+                ws=B, wsb=1 << 20, stream=None)
+    args.update(kw)
+    return fm.lib.fmlp_forward(args["x"], args["M"], args["gamma"], args["eps"], args["P"],
+                               args["T"], args["Wd"], args["d"], args["I"], args["res"],
+                               args["out"], args["ws"], args["wsb"], args["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(x=None), dict(gamma=None), dict(P=None), dict(Wd=None), dict(out=None), dict(ws=None),
+    dict(x=MIS), dict(out=MIS), dict(res=MIS), dict(ws=MIS),
+    dict(eps=0.0), dict(eps=-1e-5), dict(eps=float("inf")), dict(eps=float("nan")),
+    dict(T=12), dict(T=0), dict(T=32), dict(d=250), dict(I=690), dict(M=-1),
+    dict(wsb=16), dict(d=40000),
+])
+def test_forward_rejects_invalid_arguments(bad):
+    assert _fwd(**bad) == fm.FMLP_ERR_INVALID_ARG
+
+
+def test_forward_m0_is_a_noop():
+    assert _fwd(M=0) == fm.FMLP_OK
+
+
+def test_pack_rejects_invalid_arguments():
+    L = fm.lib
+    assert L.fmlp_pack(None, A, 256, 688, 16, B, None) == fm.FMLP_ERR_INVALID_ARG
+    assert L.fmlp_pack(A, A + 0x100000, 256, 688, 12, B + 0x10000000, None) == fm.FMLP_ERR_INVALID_ARG
+    assert L.fmlp_pack(A, A + 0x100000, 256, 688, 32, B + 0x10000000, None) == fm.FMLP_ERR_INVALID_ARG
+    # output overlapping an input
+    assert L.fmlp_pack(A, A + 0x100000, 256, 688, 16, A + 0x80, None) == fm.FMLP_ERR_INVALID_ARG
+    assert L.fmlp_pack(A, A + 0x100000, 250, 688, 16, B + 0x10000000, None) == fm.FMLP_ERR_INVALID_ARG
+
+
+def test_stage_calls_reject_invalid_arguments():
+    L = fm.lib
+    assert L.fmlp_gate_up_swiglu(A, 4, A, 1e-5, A, 16, 256, 688, None, B, 1 << 20, None) == \
+        fm.FMLP_ERR_INVALID_ARG
+    assert L.fmlp_gate_up_swiglu(A, 4, A, 0.0, A, 16, 256, 688, A, B, 1 << 20, None) == \
+        fm.FMLP_ERR_INVALID_ARG
+    assert L.fmlp_down_proj(A, 4, A, 256, 688, MIS, B, B, 1 << 20, None) == fm.FMLP_ERR_INVALID_ARG
+    assert L.fmlp_down_proj(A, 4, A, 256, 688, None, B, B, 8, None) == fm.FMLP_ERR_INVALID_ARG
+    assert L.fmlp_gate_up_swiglu(A, 0, A, 1e-5, A, 16, 256, 688, A, B, 1 << 20, None) == fm.FMLP_OK
+    assert L.fmlp_down_proj(A, 0, A, 256, 688, None, B, B, 1 << 20, None) == fm.FMLP_OK
+    assert L.fmlp_device_status(None, None) == fm.FMLP_ERR_INVALID_ARG
+
+
+def test_binding_checks_dtypes():
+    import torch
+    x = torch.zeros(2, 8, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        fm.fmlp_pack(x, x, 8, x)

@@ -1,0 +1,48 @@
+"""Host-side logic of bench.py: algorithmic byte counts and the reference arm's JSON line."""
+
+import json
+import subprocess
+import sys
+import os
+
+import bench
+import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_bytes_match_the_workload_table():
+    # 6dI weights + 2Md x + 2d gamma + 4Md f32 out
+    assert bench.algorithmic_bytes(1, 3072, 8192) == 151_019_520
+    assert round(bench.algorithmic_bytes(1, 4096, 14336) / 1e6, 2) == 352.35
+    assert bench.algorithmic_bytes(32, 4096, 14336) == 353_116_160
+    assert round(bench.algorithmic_bytes(128, 8192, 28672) / 1e6, 2) == 1415.59
+    assert bench.algorithmic_bytes(2, 8, 8, residual=True) - bench.algorithmic_bytes(2, 8, 8) == 32
+    assert bench.gateup_bytes(1, 3072, 8192) == 4 * 3072 * 8192 + 2 * 3072 + 2 * 3072 + 2 * 8192
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "3", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["config"]["workload"] == "tiny"
+
+
+def test_reference_arm_nonzero_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "3", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_warmup_floor():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--warmup", "2"], capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert out.returncode != 0

@@ -1,0 +1,292 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Bars (from the method's accuracy statement for this build):
+  * the MLP output: normwise relative error <= 2e-3 and per-element error
+    <= 1e-2 * max|O_ref| against the binary64 oracle;
+  * diagnostic, tighter: against the oracle with its intermediate rounded to
+    bf16 (the precision the fused design stores), normwise <= 2e-4 -- what is
+    left is f32 accumulation and the few elements of a whose f32 value sits on
+    the other side of a bf16 rounding boundary;
+  * the packer: bit-exact against the oracle's permutation.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-5
+TOL_NORM, TOL_ELEM, TOL_TIGHT = 2e-3, 1e-2, 2e-4
+
+
+@pytest.fixture(scope="module")
+def fm(cuda_device):
+    import token_phase_swiglu_b200 as fm
+    return fm
+
+
+def bits(t):
+    return wl.bf16_bits(t.cpu())
+
+
+def errors(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    norm = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    elem = np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-300)
+    return norm, elem
+
+
+def assert_parity(got, ref, ref_tight=None):
+    norm, elem = errors(got, ref)
+    assert norm <= TOL_NORM, f"normwise {norm:.3e}"
+    assert elem <= TOL_ELEM, f"per-element {elem:.3e}"
+    if ref_tight is not None:
+        nt, _ = errors(got, ref_tight)
+        assert nt <= TOL_TIGHT, f"normwise vs bf16-intermediate oracle {nt:.3e}"
+    return norm, elem
+
+
+def run_forward(fm, p, T=16, residual=False, stream=None):
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in p.items()}
+    M, d = g["x"].shape
+    I = g["W_gate"].shape[0]
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed, stream=stream)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    out = torch.full((M, d), float("nan"), dtype=torch.float32, device=dev)
+    fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, T, g["W_down"], out, ws,
+                    residual=g["residual"] if residual else None, stream=stream)
+    torch.cuda.synchronize()
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+    return out.cpu().double().numpy()
+
+
+def oracle_out(p, rows=None, residual=False, intermediate=None):
+    sel = slice(None) if rows is None else rows
+    b = {k: bits(v) for k, v in p.items()}
+    return oracle.fused_mlp_bf16(b["x"][sel], b["gamma"], EPS, b["W_gate"], b["W_up"],
+                                 b["W_down"],
+                                 residual_bits=b["residual"][sel] if residual else None,
+                                 intermediate=intermediate)
+
+
+# ----------------------------------------------------------------------------
+# a0: packer
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,I,T", [(256, 688, 16), (256, 688, 8), (64, 64, 64), (520, 96, 8),
+                                   (3072, 8192, 16), (4096, 14336, 32), (8, 8, 8)])
+def test_pack_bit_exact(fm, d, I, T):
+    dev = torch.device("cuda:0")
+    Wg = wl.normal_bf16(1, 2, (I, d), std=0.02)
+    Wu = wl.normal_bf16(1, 3, (I, d), std=0.02)
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(Wg.to(dev), Wu.to(dev), T, packed)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(packed), oracle.pack_gate_up(bits(Wg), bits(Wu), T))
+
+
+# ----------------------------------------------------------------------------
+# a1-a6 at small, ragged sizes (several tiles, tails, every token-chunk shape)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 7, 9, 16])
+@pytest.mark.parametrize("d,I", [(256, 688), (520, 328), (64, 16), (1032, 2064)])
+def test_forward_small(fm, M, d, I):
+    p = wl.make_problem(M, d, I, sigma=0.05, seed=M * 7 + d, residual=True)
+    for residual in (False, True):
+        got = run_forward(fm, p, T=8 if I % 16 else 16, residual=residual)
+        ref = oracle_out(p, residual=residual)
+        tight = oracle_out(p, residual=residual, intermediate="bf16")
+        assert_parity(got, ref, tight)
+
+
+@pytest.mark.parametrize("T", [8, 16, 32, 64])
+def test_forward_tile_sizes(fm, T):
+    p = wl.make_problem(3, 512, 1024, sigma=0.04, seed=T)
+    got = run_forward(fm, p, T=T)
+    assert_parity(got, oracle_out(p), oracle_out(p, intermediate="bf16"))
+
+
+def test_gate_up_intermediate(fm):
+    M, d, I, T = 5, 768, 1200, 16
+    p = wl.make_problem(M, d, I, sigma=0.04, seed=11)
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in p.items()}
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    a = torch.empty(M, I, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_gate_up_swiglu(g["x"], g["gamma"], EPS, packed, T, a, ws)
+    torch.cuda.synchronize()
+    b = {k: bits(v) for k, v in p.items()}
+    h = oracle.rmsnorm(oracle.decode_bf16(b["x"]), oracle.decode_bf16(b["gamma"]), EPS)
+    a_ref = oracle.swiglu_intermediate(h, oracle.decode_bf16(b["W_gate"]),
+                                       oracle.decode_bf16(b["W_up"]))
+    a_got = oracle.decode_bf16(bits(a))
+    # one rounding to bf16: normwise within the bf16 half-ulp budget
+    norm, _ = errors(a_got, a_ref)
+    assert norm <= 2.5e-3
+    # and almost every element is exactly the correctly rounded value
+    a_rn = oracle.round_to_bf16(a_ref)
+    mismatch = a_got != a_rn
+    assert mismatch.mean() < 1e-2
+    # the rest are one bf16 step away (a bf16 value in [2^(e-1), 2^e) has step 2^(e-8))
+    ulp = np.ldexp(1.0, np.frexp(a_rn[mismatch])[1] - 8)
+    assert np.all(np.abs(a_got[mismatch] - a_rn[mismatch]) <= ulp * 1.0001)
+
+
+def test_down_proj_alone(fm):
+    M, d, I = 6, 1024, 3000
+    dev = torch.device("cuda:0")
+    a = wl.normal_bf16(5, 0, (M, I))
+    Wd = wl.normal_bf16(5, 4, (d, I), std=0.02)
+    res = wl.normal_bf16(5, 5, (M, d))
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    for with_res in (False, True):
+        out = torch.empty(M, d, dtype=torch.float32, device=dev)
+        fm.fmlp_down_proj(a.to(dev), Wd.to(dev), out, ws, residual=res.to(dev) if with_res else None)
+        torch.cuda.synchronize()
+        ref = oracle.decode_bf16(bits(a)) @ oracle.decode_bf16(bits(Wd)).T
+        if with_res:
+            ref = ref + oracle.decode_bf16(bits(res))
+        norm, _ = errors(out.cpu().double().numpy(), ref)
+        assert norm <= 1e-5
+
+
+# ----------------------------------------------------------------------------
+# Full-size workloads (the shapes the benchmark times).  Token rows are
+# independent, so the biggest batch is checked on a sample of rows.
+# ----------------------------------------------------------------------------
+
+FULL = [
+    ("tiny", 0, None),
+    ("phi3_decode", 0, None),
+    ("phi3_decode", 31, None),
+    ("llama8b_decode_m1", 0, None),
+    ("llama8b_decode_m8", 0, None),
+    ("llama8b_decode_m32", 0, None),
+    ("llama70b_verify", 0, None),
+    ("llama8b_prefill", 0, [0, 1, 2, 255, 1000, 1023, 1024, 2047]),
+]
+
+
+@pytest.mark.parametrize("name,seed,rows", FULL, ids=[f"{n}-s{s}" for n, s, _ in FULL])
+def test_forward_full_size(fm, name, seed, rows):
+    w = wl.WORKLOADS[name]
+    p = wl.make_problem(w.M, w.d, w.I, sigma=w.sigma, seed=seed)
+    got = run_forward(fm, p, T=16)
+    if rows is not None:
+        got = got[rows]
+    ref = oracle_out(p, rows=rows)
+    tight = oracle_out(p, rows=rows, intermediate="bf16")
+    norm, elem = assert_parity(got, ref, tight)
+    print(f"{name} seed {seed}: normwise {norm:.3e} per-element {elem:.3e}")
+
+
+# ----------------------------------------------------------------------------
+# Edge cases
+# ----------------------------------------------------------------------------
+
+def test_m0_is_a_noop(fm):
+    dev = torch.device("cuda:0")
+    d, I = 256, 688
+    x = torch.empty(0, d, dtype=torch.bfloat16, device=dev)
+    gamma = torch.ones(d, dtype=torch.bfloat16, device=dev)
+    packed = torch.zeros(2 * I, d, dtype=torch.bfloat16, device=dev)
+    Wd = torch.zeros(d, I, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(0, d, dtype=torch.float32, device=dev)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(0, d, I), dtype=torch.uint8, device=dev)
+    fm.fmlp_forward(x, gamma, EPS, packed, 16, Wd, out, ws)
+    torch.cuda.synchronize()
+
+
+def test_zero_rows_and_zero_weights(fm):
+    p = wl.make_problem(4, 256, 688, seed=3, residual=True)
+    p["x"][2].zero_()
+    got = run_forward(fm, p, residual=True)
+    # a zero token row gives h = 0, so the output row is exactly the residual row
+    assert np.array_equal(got[2], p["residual"][2].double().numpy())
+    assert_parity(got, oracle_out(p, residual=True))
+    # zero gate weights: SiLU(0) = 0 makes the MLP output exactly zero
+    p["W_gate"].zero_()
+    got = run_forward(fm, p)
+    assert np.all(got == 0.0)
+
+
+def test_saturating_gate(fm):
+    # large weights drive |g| past 88, where exp(-g) overflows (SiLU -> -0) or SiLU(g) = g
+    p = wl.make_problem(3, 512, 256, sigma=1.0, seed=4)
+    b = {k: bits(v) for k, v in p.items()}
+    h = oracle.rmsnorm(oracle.decode_bf16(b["x"]), oracle.decode_bf16(b["gamma"]), EPS)
+    g = h @ oracle.decode_bf16(b["W_gate"]).T
+    assert g.min() < -88 and g.max() > 88
+    got = run_forward(fm, p)
+    assert np.all(np.isfinite(got))
+    assert_parity(got, oracle_out(p), oracle_out(p, intermediate="bf16"))
+
+
+def test_large_and_tiny_inputs(fm):
+    # RMSNorm removes the scale of x: 2^k x gives the same output up to eps drift
+    p = wl.make_problem(2, 256, 688, seed=5)
+    base = run_forward(fm, p)
+    for k in (-6, 8):
+        q = dict(p)
+        q["x"] = (p["x"].double() * 2.0 ** k).to(torch.bfloat16)
+        got = run_forward(fm, q)
+        assert_parity(got, oracle_out(q))
+        assert errors(got, base)[0] < 1e-3
+
+
+def test_side_stream_and_workspace_reuse(fm):
+    p = wl.make_problem(3, 256, 688, seed=6, residual=True)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        got = run_forward(fm, p, residual=True, stream=s)
+    assert_parity(got, oracle_out(p, residual=True))
+    # same workspace, different M: workspace must only be big enough
+    dev = torch.device("cuda:0")
+    d, I, T = 256, 688, 16
+    g = {k: v.to(dev) for k, v in p.items()}
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(3, d, I), dtype=torch.uint8, device=dev)
+    for M in (3, 1, 2, 3):
+        out = torch.empty(M, d, dtype=torch.float32, device=dev)
+        fm.fmlp_forward(g["x"][:M].contiguous(), g["gamma"], EPS, packed, T, g["W_down"], out, ws)
+        torch.cuda.synchronize()
+        assert_parity(out.cpu().double().numpy(), oracle_out(p, rows=slice(0, M)))
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+
+
+def test_invalid_arguments_raise(fm):
+    dev = torch.device("cuda:0")
+    d, I = 256, 688
+    x = torch.zeros(2, d, dtype=torch.bfloat16, device=dev)
+    gamma = torch.ones(d, dtype=torch.bfloat16, device=dev)
+    packed = torch.zeros(2 * I, d, dtype=torch.bfloat16, device=dev)
+    Wd = torch.zeros(d, I, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(2, d, dtype=torch.float32, device=dev)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(2, d, I), dtype=torch.uint8, device=dev)
+    with pytest.raises(fm.FmlpError) as e:
+        fm.fmlp_forward(x, gamma, 0.0, packed, 16, Wd, out, ws)
+    assert e.value.status == fm.FMLP_ERR_INVALID_ARG
+    with pytest.raises(fm.FmlpError):
+        fm.fmlp_forward(x, gamma, EPS, packed, 16, Wd, out, ws[:64])
+    mis = torch.zeros(2 * d + 8, dtype=torch.bfloat16, device=dev)[4:4 + 2 * d].view(2, d)
+    with pytest.raises(fm.FmlpError):
+        fm.fmlp_forward(mis, gamma, EPS, packed, 16, Wd, out, ws)
+    torch.cuda.synchronize()
+
+
+def test_loaded_library_is_in_tree(fm):
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    assert os.path.commonpath([fm.LIB_PATH, root]) == root
+    with open("/proc/self/maps") as f:
+        assert fm.LIB_PATH in f.read()

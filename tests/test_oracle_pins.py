@@ -235,6 +235,22 @@ def pin_saturated_gate_is_bilinear(o):
     assert np.max(np.abs(got_neg)) < 1e-20
 
 
+def pin_swiglu_intermediate(o):
+    # a is what gated_mlp feeds the down projection: W_down = I recovers it
+    rng = np.random.default_rng(11)
+    M, d, I = 2, 6, 6
+    h = _bf16_values(rng, (M, d))
+    Wg, Wu = _bf16_values(rng, (I, d), 0.5), _bf16_values(rng, (I, d), 0.5)
+    a = o.swiglu_intermediate(h, Wg, Wu)
+    assert a.shape == (M, I)
+    np.testing.assert_allclose(o.gated_mlp(h, Wg, Wu, np.eye(I)), a, rtol=1e-15, atol=0)
+    for m in range(M):
+        for i in range(I):
+            g = float(sum(Fraction(Wg[i, k]) * Fraction(h[m, k]) for k in range(d)))
+            u = float(sum(Fraction(Wu[i, k]) * Fraction(h[m, k]) for k in range(d)))
+            assert abs(a[m, i] - g / (1 + math.exp(-g)) * u) <= 1e-14 * (1 + abs(a[m, i]))
+
+
 def pin_intermediate_rounding(o):
     rng = np.random.default_rng(6)
     M, d, I = 2, 16, 12
@@ -313,7 +329,8 @@ def pin_bf16_entry_decodes(o):
 
 PINS = [pin_decode_bf16_exhaustive, pin_round_to_bf16, pin_rms_inv_vs_norm,
         pin_rmsnorm_scale_invariance, pin_silu, pin_closed_form_d1_I1, pin_zero_invariants,
-        pin_bruteforce_tiny, pin_saturated_gate_is_bilinear, pin_intermediate_rounding,
+        pin_bruteforce_tiny, pin_saturated_gate_is_bilinear, pin_swiglu_intermediate,
+        pin_intermediate_rounding,
         pin_interleave_golden, pin_interleave_is_permutation, pin_packed_forward_equals_plain,
         pin_bf16_entry_decodes]
 
@@ -324,7 +341,8 @@ def test_oracle_pin(pin):
 
 
 def test_package_exports_are_the_pinned_functions():
-    for name in ["decode_bf16", "round_to_bf16", "rms_inv", "rmsnorm", "silu", "gated_mlp",
+    for name in ["decode_bf16", "round_to_bf16", "rms_inv", "rmsnorm", "silu",
+                 "swiglu_intermediate", "gated_mlp",
                  "fused_mlp", "interleaved_rows", "pack_gate_up", "unpack_gate_up",
                  "fused_mlp_packed", "fused_mlp_bf16"]:
         assert getattr(oracle, name) is getattr(ofm, name)

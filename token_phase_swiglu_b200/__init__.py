@@ -1,0 +1,164 @@
+"""Python binding of libfmlp.so, the B200 fused gated-MLP library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/fmlp.h``.  Tensors are torch
+CUDA tensors (torch provides device memory and streams); the functions pass
+their device pointers and sizes through ctypes and raise ``FmlpError`` on any
+status other than FMLP_OK.  There is no fallback: if the shared library has
+not been built, importing this package raises ImportError.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "FmlpError", "FMLP_OK", "FMLP_ERR_INVALID_ARG", "FMLP_ERR_UNSUPPORTED", "FMLP_ERR_CUDA",
+    "FMLP_ERR_TIMEOUT", "LIB_PATH", "lib", "fmlp_pack", "fmlp_workspace_bytes", "fmlp_forward",
+    "fmlp_gate_up_swiglu", "fmlp_down_proj", "fmlp_device_status", "fmlp_status_string",
+    "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "EXPORTED_SYMBOLS",
+]
+
+FMLP_OK, FMLP_ERR_INVALID_ARG, FMLP_ERR_UNSUPPORTED, FMLP_ERR_CUDA, FMLP_ERR_TIMEOUT = range(5)
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfmlp.so")
+
+_i64, _sz, _vp, _int, _f32 = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+
+# name -> (restype, argtypes); mirrors include/fmlp.h
+_SIGNATURES = {
+    "fmlp_pack": (_int, [_vp, _vp, _i64, _i64, _int, _vp, _vp]),
+    "fmlp_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "fmlp_forward": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "fmlp_gate_up_swiglu": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "fmlp_down_proj": (_int, [_vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "fmlp_device_status": (_int, [_vp, _vp]),
+    "fmlp_status_string": (ctypes.c_char_p, [_int]),
+    "fmlp_last_cuda_error": (_int, []),
+    "fmlp_kernel_launch_count": (ctypes.c_uint64, []),
+}
+EXPORTED_SYMBOLS = tuple(_SIGNATURES)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'` "
+            "(nvcc, sm_100a). There is no non-CUDA implementation.")
+    handle = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
+
+
+lib = _load()
+
+
+class FmlpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.fmlp_status_string(status).decode()
+        if status == FMLP_ERR_CUDA:
+            msg += f" (cudaError {lib.fmlp_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != FMLP_OK:
+        raise FmlpError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libfmlp must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _bf16(t, name):
+    if t is not None and t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+
+
+def fmlp_status_string(status: int) -> str:
+    return lib.fmlp_status_string(status).decode()
+
+
+def fmlp_last_cuda_error() -> int:
+    return lib.fmlp_last_cuda_error()
+
+
+def fmlp_kernel_launch_count() -> int:
+    return int(lib.fmlp_kernel_launch_count())
+
+
+def fmlp_workspace_bytes(M: int, d: int, I: int) -> int:
+    return int(lib.fmlp_workspace_bytes(M, d, I))
+
+
+def fmlp_pack(W_gate, W_up, tile_T: int, packed, stream=None) -> None:
+    """packed [2I x d] <- rows of W_gate / W_up [I x d] interleaved at tile tile_T."""
+    _bf16(W_gate, "W_gate"); _bf16(W_up, "W_up"); _bf16(packed, "packed")
+    I, d = W_gate.shape
+    _check(lib.fmlp_pack(_ptr(W_gate), _ptr(W_up), d, I, tile_T, _ptr(packed), _stream(stream)),
+           "fmlp_pack")
+
+
+def fmlp_forward(x, gamma, eps: float, packed, tile_T: int, W_down, out, workspace,
+                 residual=None, stream=None) -> None:
+    """out [M x d] (f32) <- RMSNorm + gated MLP (+ residual) of x [M x d]."""
+    for t, n in ((x, "x"), (gamma, "gamma"), (packed, "packed"), (W_down, "W_down"),
+                 (residual, "residual")):
+        _bf16(t, n)
+    M, d = x.shape
+    I = W_down.shape[1]
+    _check(lib.fmlp_forward(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T, _ptr(W_down),
+                            d, I, _ptr(residual), _ptr(out), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fmlp_forward")
+
+
+def fmlp_gate_up_swiglu(x, gamma, eps: float, packed, tile_T: int, a, workspace,
+                        stream=None) -> None:
+    """a [M x I] (bf16) <- SiLU(gate) * up of RMSNorm(x) against packed gate/up rows."""
+    for t, n in ((x, "x"), (gamma, "gamma"), (packed, "packed"), (a, "a")):
+        _bf16(t, n)
+    M, d = x.shape
+    I = a.shape[1]
+    _check(lib.fmlp_gate_up_swiglu(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T, d, I,
+                                   _ptr(a), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fmlp_gate_up_swiglu")
+
+
+def fmlp_down_proj(a, W_down, out, workspace, residual=None, stream=None) -> None:
+    """out [M x d] (f32) <- a [M x I] W_down^T (+ residual)."""
+    for t, n in ((a, "a"), (W_down, "W_down"), (residual, "residual")):
+        _bf16(t, n)
+    M, I = a.shape
+    d = W_down.shape[0]
+    _check(lib.fmlp_down_proj(_ptr(a), M, _ptr(W_down), d, I, _ptr(residual), _ptr(out),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)),
+           "fmlp_down_proj")
+
+
+def fmlp_device_status(workspace, stream=None) -> int:
+    """Synchronise, read and clear the workspace's device status word; returns the status."""
+    return int(lib.fmlp_device_status(_ptr(workspace), _stream(stream)))

@@ -1,0 +1,213 @@
+// C ABI of libfmlp.so: argument validation, path selection and launches.
+// The contract (layouts, ownership, errors) is documented in include/fmlp.h.
+#include "fmlp.h"
+#include "internal.h"
+
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+namespace fmlp {
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_info[kMaxDevices];
+std::once_flag g_once[kMaxDevices];
+cudaError_t g_info_err[kMaxDevices];
+
+constexpr int64_t kMaxD = 32768;
+constexpr int64_t kMaxI = 131072;
+
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+fmlp_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return FMLP_ERR_CUDA;
+}
+
+bool sizes_ok(int64_t M, int64_t d, int64_t I) {
+  return M >= 0 && d > 0 && I > 0 && d % 8 == 0 && I % 8 == 0 && d <= kMaxD && I <= kMaxI &&
+         M <= (int64_t)1 << 24;
+}
+
+bool tile_ok(int T, int64_t I) { return T > 0 && T % 8 == 0 && I % T == 0; }
+
+bool eps_ok(float eps) { return std::isfinite(eps) && eps > 0.f; }
+
+// Resolve the current device's cached attributes and check it is sm_100.
+fmlp_status device_for_launch(const DeviceInfo** info) {
+  cudaError_t e = current_device_info(info);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if ((*info)->cc_major != 10) return FMLP_ERR_UNSUPPORTED;
+  return FMLP_OK;
+}
+
+}  // namespace
+
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+cudaError_t current_device_info(const DeviceInfo** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_once[dev], [dev] {
+    DeviceInfo& di = g_info[dev];
+    di.device = dev;
+    cudaError_t err = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (err == cudaSuccess)
+      err = cudaDeviceGetAttribute(&di.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (err == cudaSuccess)
+      err = cudaDeviceGetAttribute(&di.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (err == cudaSuccess)
+      err = cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                   dev);
+    g_info_err[dev] = err;
+  });
+  *out = &g_info[dev];
+  return g_info_err[dev];
+}
+
+WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
+  (void)d;
+  WorkspaceLayout L;
+  size_t off = 0;
+  L.status = off;
+  off += 256;
+  L.a = off;
+  off += align256((size_t)M * (size_t)I * 2);
+  L.total = off;
+  return L;
+}
+
+}  // namespace fmlp
+
+using namespace fmlp;
+
+extern "C" {
+
+const char* fmlp_status_string(fmlp_status s) {
+  switch (s) {
+    case FMLP_OK: return "FMLP_OK";
+    case FMLP_ERR_INVALID_ARG: return "FMLP_ERR_INVALID_ARG: invalid argument";
+    case FMLP_ERR_UNSUPPORTED: return "FMLP_ERR_UNSUPPORTED: request outside the implemented kernels";
+    case FMLP_ERR_CUDA: return "FMLP_ERR_CUDA: a CUDA call or launch failed";
+    case FMLP_ERR_TIMEOUT: return "FMLP_ERR_TIMEOUT: a bounded device wait expired";
+  }
+  return "unknown fmlp_status";
+}
+
+int fmlp_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t fmlp_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I) {
+  if (!sizes_ok(M, d, I)) return 0;
+  return workspace_layout(M, d, I).total;
+}
+
+fmlp_status fmlp_pack(const void* W_gate, const void* W_up, int64_t d, int64_t I, int tile_T,
+                      void* packed, void* stream) {
+  if (!W_gate || !W_up || !packed) return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(packed)) return FMLP_ERR_INVALID_ARG;
+  if (!sizes_ok(0, d, I) || !tile_ok(tile_T, I)) return FMLP_ERR_INVALID_ARG;
+  // the output must not overlap either input
+  const uintptr_t p0 = (uintptr_t)packed, p1 = p0 + (uintptr_t)(2 * I * d * 2);
+  const uintptr_t in_bytes = (uintptr_t)(I * d * 2);
+  for (const void* src : {W_gate, W_up}) {
+    const uintptr_t s0 = (uintptr_t)src, s1 = s0 + in_bytes;
+    if (s0 < p1 && p0 < s1) return FMLP_ERR_INVALID_ARG;
+  }
+  const DeviceInfo* dev = nullptr;
+  fmlp_status st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  cudaError_t e = launch_pack(W_gate, W_up, d, I, tile_T, packed, (cudaStream_t)stream);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
+static fmlp_status check_common(int64_t M, int64_t d, int64_t I, void* workspace,
+                                size_t workspace_bytes) {
+  if (!sizes_ok(M, d, I)) return FMLP_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace)) return FMLP_ERR_INVALID_ARG;
+  if (workspace_bytes < workspace_layout(M, d, I).total) return FMLP_ERR_INVALID_ARG;
+  return FMLP_OK;
+}
+
+fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* gamma, float eps,
+                                const void* packed_Wgu, int tile_T, int64_t d, int64_t I,
+                                void* a, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
+  if (st != FMLP_OK) return st;
+  if (!x || !gamma || !packed_Wgu || !a) return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed_Wgu) || !aligned16(a))
+    return FMLP_ERR_INVALID_ARG;
+  if (!eps_ok(eps) || !tile_ok(tile_T, I)) return FMLP_ERR_INVALID_ARG;
+  if (M == 0) return FMLP_OK;
+  const DeviceInfo* dev = nullptr;
+  st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  cudaError_t e = launch_gateup_gemv(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, *dev,
+                                     (cudaStream_t)stream);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
+fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t d, int64_t I,
+                           const void* residual, float* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
+  if (st != FMLP_OK) return st;
+  if (!a || !W_down || !out) return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(W_down) || !aligned16(out)) return FMLP_ERR_INVALID_ARG;
+  if (residual && !aligned16(residual)) return FMLP_ERR_INVALID_ARG;
+  if (M == 0) return FMLP_OK;
+  const DeviceInfo* dev = nullptr;
+  st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  cudaError_t e = launch_down_gemv(a, M, W_down, d, I, residual, out, *dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
+fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
+                         const void* packed_Wgu, int tile_T, const void* W_down, int64_t d,
+                         int64_t I, const void* residual, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
+  if (st != FMLP_OK) return st;
+  if (!x || !gamma || !packed_Wgu || !W_down || !out) return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed_Wgu) || !aligned16(W_down) ||
+      !aligned16(out))
+    return FMLP_ERR_INVALID_ARG;
+  if (residual && !aligned16(residual)) return FMLP_ERR_INVALID_ARG;
+  if (!eps_ok(eps) || !tile_ok(tile_T, I)) return FMLP_ERR_INVALID_ARG;
+  if (M == 0) return FMLP_OK;
+  const DeviceInfo* dev = nullptr;
+  st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  const WorkspaceLayout L = workspace_layout(M, d, I);
+  void* a = (char*)workspace + L.a;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_gateup_gemv(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, *dev, s);
+  if (e == cudaSuccess) e = launch_down_gemv(a, M, W_down, d, I, residual, out, *dev, s);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
+fmlp_status fmlp_device_status(void* workspace, void* stream) {
+  if (!workspace || !aligned16(workspace)) return FMLP_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && word != 0) {
+    e = cudaMemsetAsync(workspace, 0, sizeof(word), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  return word & kStatusTimeout ? FMLP_ERR_TIMEOUT : FMLP_OK;
+}
+
+}  // extern "C"
