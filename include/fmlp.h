@@ -30,8 +30,9 @@
  *     CUDA error code is kept for fmlp_last_cuda_error()).  There is no CPU
  *     fallback: without a usable sm_100 device every compute call fails.
  *   - Sizes: d (hidden) and I (intermediate) must be positive multiples of 8
- *     (rows are whole 16-byte vectors), d <= 32768, I <= 131072.  M (token
- *     rows) may be 0, which is a no-op.
+ *     (rows are whole 16-byte vectors), d <= 32768, I <= 65536.  M (token
+ *     rows) may be 0, which is a no-op; then the pointers to M-row tensors
+ *     (x, a, out, residual) may be NULL.
  */
 #ifndef FMLP_H
 #define FMLP_H
@@ -79,9 +80,10 @@ FMLP_API fmlp_status fmlp_pack(const void* W_gate, const void* W_up, int64_t d, 
 /*
  * fmlp_workspace_bytes -- bytes of device workspace fmlp_forward needs for
  * (M, d, I).  The workspace holds a device status word, the bf16
- * intermediate a [M x I] and per-path scratch.  A workspace must be
- * zero-filled once before its first use; the library leaves its control
- * words at zero after every call.  Returns 0 for invalid sizes.
+ * intermediate a [M x I] and the control words of the fused kernel's
+ * grid-wide barrier.  A workspace must be zero-filled once before its first
+ * use; the library keeps its control words consistent from call to call.
+ * Returns 0 for invalid sizes.
  */
 FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
 
@@ -134,7 +136,9 @@ FMLP_API fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down
  * fmlp_device_status -- synchronise `stream`, read the device status word in
  * `workspace` and reset it to zero.  Returns FMLP_ERR_TIMEOUT if a kernel
  * gave up a bounded wait since the last check, FMLP_OK otherwise (or
- * FMLP_ERR_CUDA / FMLP_ERR_INVALID_ARG).
+ * FMLP_ERR_CUDA / FMLP_ERR_INVALID_ARG).  After a timeout it also resets the
+ * workspace's other control words, so the workspace can be used again; no
+ * other call may be using the workspace meanwhile.
  */
 FMLP_API fmlp_status fmlp_device_status(void* workspace, void* stream);
 
@@ -143,6 +147,26 @@ FMLP_API const char* fmlp_status_string(fmlp_status status);
 
 /* The cudaError_t behind the calling thread's most recent FMLP_ERR_CUDA (0 if none). */
 FMLP_API int fmlp_last_cuda_error(void);
+
+/*
+ * fmlp_set_wait_timeout_ns -- deadline for every bounded wait inside the
+ * kernels (a stage of the shared-memory ring that never fills or drains).
+ * On expiry a kernel sets the timeout bit of its workspace status word, lets
+ * its own in-flight copies land and returns; fmlp_device_status then reports
+ * FMLP_ERR_TIMEOUT and the outputs of that call are undefined.  Process-wide;
+ * 0 restores the default of one second.  Meant for diagnosis and for testing
+ * the timeout path; normal waits last microseconds.
+ */
+FMLP_API void fmlp_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * fmlp_set_fault_injection -- testing aid.  mode != 0 makes every kernel's
+ * producer withhold its last stage of weights, so the consumers' bounded
+ * waits expire and the call ends with FMLP_ERR_TIMEOUT in the status word
+ * (no GPU fault: the kernels give up and return).  0 turns it off.
+ * Process-wide; outputs of affected calls are undefined.
+ */
+FMLP_API void fmlp_set_fault_injection(int mode);
 
 /* Kernels this library has enqueued in this process so far (all threads, all
  * devices; a launch captured into a CUDA graph counts once, at capture). */

@@ -54,6 +54,8 @@ def test_workspace_bytes():
     assert L.fmlp_workspace_bytes(1, 256, 690) == 0
     assert L.fmlp_workspace_bytes(-1, 256, 688) == 0
     assert L.fmlp_workspace_bytes(1, 65536, 688) == 0
+    assert L.fmlp_workspace_bytes(1, 4096, 65544) == 0
+    assert L.fmlp_workspace_bytes(1, 32768, 65536) > 0
     for M in (1, 7, 2048):
         assert L.fmlp_workspace_bytes(M, 4096, 14336) % 256 == 0
 

@@ -4,9 +4,13 @@ Bars (from the method's accuracy statement for this build):
   * the MLP output: normwise relative error <= 2e-3 and per-element error
     <= 1e-2 * max|O_ref| against the binary64 oracle;
   * diagnostic, tighter: against the oracle with its intermediate rounded to
-    bf16 (the precision the fused design stores), normwise <= 2e-4 -- what is
-    left is f32 accumulation and the few elements of a whose f32 value sits on
-    the other side of a bf16 rounding boundary;
+    bf16 (the precision the fused design stores).  What separates the two is
+    f32 accumulation plus the few elements of a whose f32 value lands on the
+    other side of a bf16 rounding boundary than the binary64 value (each such
+    flip is one bf16 step).  With a fraction f of flipped elements that
+    difference is about sqrt(f) times the whole bf16 rounding error of a, so
+    it must stay below TIGHT_FRAC = 0.25 of that rounding error (f <~ 6%);
+    a dropped term, a wrong scale or a misplaced row costs far more;
   * the packer: bit-exact against the oracle's permutation.
 """
 
@@ -20,7 +24,7 @@ import workloads as wl
 pytestmark = pytest.mark.gpu
 
 EPS = 1e-5
-TOL_NORM, TOL_ELEM, TOL_TIGHT = 2e-3, 1e-2, 2e-4
+TOL_NORM, TOL_ELEM, TIGHT_FRAC = 2e-3, 1e-2, 0.25
 
 
 @pytest.fixture(scope="module")
@@ -46,7 +50,9 @@ def assert_parity(got, ref, ref_tight=None):
     assert elem <= TOL_ELEM, f"per-element {elem:.3e}"
     if ref_tight is not None:
         nt, _ = errors(got, ref_tight)
-        assert nt <= TOL_TIGHT, f"normwise vs bf16-intermediate oracle {nt:.3e}"
+        rounding, _ = errors(ref_tight, ref)
+        assert nt <= TIGHT_FRAC * rounding + 1e-6, \
+            f"normwise vs bf16-intermediate oracle {nt:.3e} (bf16 rounding of a: {rounding:.3e})"
     return norm, elem
 
 
@@ -221,7 +227,7 @@ def test_zero_rows_and_zero_weights(fm):
 
 def test_saturating_gate(fm):
     # large weights drive |g| past 88, where exp(-g) overflows (SiLU -> -0) or SiLU(g) = g
-    p = wl.make_problem(3, 512, 256, sigma=1.0, seed=4)
+    p = wl.make_problem(3, 512, 256, sigma=3.0, seed=4)
     b = {k: bits(v) for k, v in p.items()}
     h = oracle.rmsnorm(oracle.decode_bf16(b["x"]), oracle.decode_bf16(b["gamma"]), EPS)
     g = h @ oracle.decode_bf16(b["W_gate"]).T
@@ -232,15 +238,19 @@ def test_saturating_gate(fm):
 
 
 def test_large_and_tiny_inputs(fm):
-    # RMSNorm removes the scale of x: 2^k x gives the same output up to eps drift
+    # RMSNorm removes the scale of x: c x gives the same output up to the eps
+    # drift, which is at most eps |1 - c^-2| / (2 mean x^2) relative in h
     p = wl.make_problem(2, 256, 688, seed=5)
     base = run_forward(fm, p)
+    ms = float((p["x"].double() ** 2).mean(dim=1).min())
     for k in (-6, 8):
+        c = 2.0 ** k
         q = dict(p)
-        q["x"] = (p["x"].double() * 2.0 ** k).to(torch.bfloat16)
+        q["x"] = (p["x"].double() * c).to(torch.bfloat16)
         got = run_forward(fm, q)
-        assert_parity(got, oracle_out(q))
-        assert errors(got, base)[0] < 1e-3
+        assert_parity(got, oracle_out(q), oracle_out(q, intermediate="bf16"))
+        drift = EPS * abs(1 - c ** -2) / (2 * ms * c * c) if c < 1 else EPS / (2 * ms)
+        assert errors(got, base)[0] < 3 * drift + 2e-4
 
 
 def test_side_stream_and_workspace_reuse(fm):
@@ -290,3 +300,64 @@ def test_loaded_library_is_in_tree(fm):
     assert os.path.commonpath([fm.LIB_PATH, root]) == root
     with open("/proc/self/maps") as f:
         assert fm.LIB_PATH in f.read()
+
+
+def test_bounded_wait_timeout_reports_and_recovers(fm):
+    """Host-controlled fault: the kernels' producers withhold their last stage,
+    so the consumers' bounded waits expire.  Each kernel flags the status
+    word, lets its in-flight copies land and returns; the context stays usable
+    and the next call, with injection off, is correct."""
+    dev = torch.device("cuda:0")
+    for M in (2, 7):   # the fused kernel, and the two-kernel path
+        p = wl.make_problem(M, 1024, 2048, seed=12)
+        g = {k: v.to(dev) for k, v in p.items()}
+        d, I, T = 1024, 2048, 16
+        packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+        fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+        ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+        out = torch.empty(M, d, dtype=torch.float32, device=dev)
+        try:
+            fm.fmlp_set_wait_timeout_ns(2_000_000)
+            fm.fmlp_set_fault_injection(1)
+            fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, T, g["W_down"], out, ws)
+            torch.cuda.synchronize()
+        finally:
+            fm.fmlp_set_fault_injection(0)
+            fm.fmlp_set_wait_timeout_ns(0)
+        assert fm.fmlp_device_status(ws) == fm.FMLP_ERR_TIMEOUT
+        assert fm.fmlp_device_status(ws) == fm.FMLP_OK       # reading clears the word
+        fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, T, g["W_down"], out, ws)
+        torch.cuda.synchronize()
+        assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+        assert_parity(out.cpu().double().numpy(), oracle_out(p))
+
+
+def test_fused_and_two_kernel_paths_agree(fm):
+    """For M <= 4 fmlp_forward runs one fused launch; the stage calls run the
+    same phases as two launches.  Same arithmetic, same order: identical bits."""
+    dev = torch.device("cuda:0")
+    for (M, d, I) in [(1, 3072, 8192), (3, 1024, 2064), (4, 256, 688)]:
+        p = wl.make_problem(M, d, I, seed=21, residual=True)
+        g = {k: v.to(dev) for k, v in p.items()}
+        packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+        fm.fmlp_pack(g["W_gate"], g["W_up"], 16, packed)
+        ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+        fused = torch.empty(M, d, dtype=torch.float32, device=dev)
+        fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, 16, g["W_down"], fused, ws,
+                        residual=g["residual"])
+        a = torch.empty(M, I, dtype=torch.bfloat16, device=dev)
+        two = torch.empty(M, d, dtype=torch.float32, device=dev)
+        fm.fmlp_gate_up_swiglu(g["x"], g["gamma"], EPS, packed, 16, a, ws)
+        fm.fmlp_down_proj(a, g["W_down"], two, ws, residual=g["residual"])
+        torch.cuda.synchronize()
+        assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+        assert torch.equal(fused, two)
+
+
+@pytest.mark.parametrize("M,d,I", [(1, 32768, 64), (4, 32768, 64), (1, 64, 65536), (3, 64, 65536),
+                                   (2, 8, 8)])
+def test_maximum_and_minimum_sizes(fm, M, d, I):
+    p = wl.make_problem(M, d, I, sigma=0.05, seed=13, residual=True)
+    got = run_forward(fm, p, T=8, residual=True)
+    assert_parity(got, oracle_out(p, residual=True), oracle_out(p, residual=True,
+                                                               intermediate="bf16"))

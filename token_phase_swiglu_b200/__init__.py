@@ -19,7 +19,8 @@ __all__ = [
     "FmlpError", "FMLP_OK", "FMLP_ERR_INVALID_ARG", "FMLP_ERR_UNSUPPORTED", "FMLP_ERR_CUDA",
     "FMLP_ERR_TIMEOUT", "LIB_PATH", "lib", "fmlp_pack", "fmlp_workspace_bytes", "fmlp_forward",
     "fmlp_gate_up_swiglu", "fmlp_down_proj", "fmlp_device_status", "fmlp_status_string",
-    "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "EXPORTED_SYMBOLS",
+    "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "fmlp_set_wait_timeout_ns", "fmlp_set_fault_injection",
+    "EXPORTED_SYMBOLS",
 ]
 
 FMLP_OK, FMLP_ERR_INVALID_ARG, FMLP_ERR_UNSUPPORTED, FMLP_ERR_CUDA, FMLP_ERR_TIMEOUT = range(5)
@@ -39,6 +40,8 @@ _SIGNATURES = {
     "fmlp_status_string": (ctypes.c_char_p, [_int]),
     "fmlp_last_cuda_error": (_int, []),
     "fmlp_kernel_launch_count": (ctypes.c_uint64, []),
+    "fmlp_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
+    "fmlp_set_fault_injection": (None, [_int]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -106,6 +109,16 @@ def fmlp_last_cuda_error() -> int:
 
 def fmlp_kernel_launch_count() -> int:
     return int(lib.fmlp_kernel_launch_count())
+
+
+def fmlp_set_wait_timeout_ns(ns: int) -> None:
+    """Deadline of the kernels' bounded waits (0 = default, one second)."""
+    lib.fmlp_set_wait_timeout_ns(int(ns))
+
+
+def fmlp_set_fault_injection(mode: int) -> None:
+    """Testing aid: nonzero makes kernels withhold their last stage (bounded waits expire)."""
+    lib.fmlp_set_fault_injection(int(mode))
 
 
 def fmlp_workspace_bytes(M: int, d: int, I: int) -> int:

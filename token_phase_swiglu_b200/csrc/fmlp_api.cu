@@ -12,6 +12,9 @@ namespace {
 
 thread_local int g_last_cuda_error = 0;
 std::atomic<uint64_t> g_launches{0};
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;  // 1 s
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_fault{0};
 
 constexpr int kMaxDevices = 64;
 DeviceInfo g_info[kMaxDevices];
@@ -19,10 +22,12 @@ std::once_flag g_once[kMaxDevices];
 cudaError_t g_info_err[kMaxDevices];
 
 constexpr int64_t kMaxD = 32768;
-constexpr int64_t kMaxI = 131072;
+constexpr int64_t kMaxI = 65536;
 
 inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
-inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }  // NULL passes
+
+inline uint32_t* status_word(void* workspace) { return (uint32_t*)workspace; }
 
 fmlp_status cuda_fail(cudaError_t e) {
   g_last_cuda_error = (int)e;
@@ -49,6 +54,10 @@ fmlp_status device_for_launch(const DeviceInfo** info) {
 }  // namespace
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+uint64_t wait_timeout_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
+int fault_injection() { return g_fault.load(std::memory_order_relaxed); }
 
 cudaError_t current_device_info(const DeviceInfo** out) {
   int dev = -1;
@@ -77,6 +86,7 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
   WorkspaceLayout L;
   size_t off = 0;
   L.status = off;
+  L.barrier = off + 64;
   off += 256;
   L.a = off;
   off += align256((size_t)M * (size_t)I * 2);
@@ -104,6 +114,12 @@ const char* fmlp_status_string(fmlp_status s) {
 int fmlp_last_cuda_error(void) { return g_last_cuda_error; }
 
 uint64_t fmlp_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void fmlp_set_wait_timeout_ns(uint64_t ns) {
+  g_wait_ns.store(ns ? ns : kDefaultWaitNs, std::memory_order_relaxed);
+}
+
+void fmlp_set_fault_injection(int mode) { g_fault.store(mode ? 1 : 0, std::memory_order_relaxed); }
 
 size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I) {
   if (!sizes_ok(M, d, I)) return 0;
@@ -143,7 +159,8 @@ fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* gamma, flo
                                 void* stream) {
   fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
   if (st != FMLP_OK) return st;
-  if (!x || !gamma || !packed_Wgu || !a) return FMLP_ERR_INVALID_ARG;
+  if (!gamma || !packed_Wgu) return FMLP_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !a)) return FMLP_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed_Wgu) || !aligned16(a))
     return FMLP_ERR_INVALID_ARG;
   if (!eps_ok(eps) || !tile_ok(tile_T, I)) return FMLP_ERR_INVALID_ARG;
@@ -151,8 +168,8 @@ fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* gamma, flo
   const DeviceInfo* dev = nullptr;
   st = device_for_launch(&dev);
   if (st != FMLP_OK) return st;
-  cudaError_t e = launch_gateup_gemv(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, *dev,
-                                     (cudaStream_t)stream);
+  cudaError_t e = launch_gateup_stream(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a,
+                                       status_word(workspace), *dev, (cudaStream_t)stream);
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
 }
 
@@ -161,14 +178,16 @@ fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t
                            size_t workspace_bytes, void* stream) {
   fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
   if (st != FMLP_OK) return st;
-  if (!a || !W_down || !out) return FMLP_ERR_INVALID_ARG;
-  if (!aligned16(a) || !aligned16(W_down) || !aligned16(out)) return FMLP_ERR_INVALID_ARG;
-  if (residual && !aligned16(residual)) return FMLP_ERR_INVALID_ARG;
+  if (!W_down) return FMLP_ERR_INVALID_ARG;
+  if (M > 0 && (!a || !out)) return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(W_down) || !aligned16(out) || !aligned16(residual))
+    return FMLP_ERR_INVALID_ARG;
   if (M == 0) return FMLP_OK;
   const DeviceInfo* dev = nullptr;
   st = device_for_launch(&dev);
   if (st != FMLP_OK) return st;
-  cudaError_t e = launch_down_gemv(a, M, W_down, d, I, residual, out, *dev, (cudaStream_t)stream);
+  cudaError_t e = launch_down_stream(a, M, W_down, d, I, residual, out, status_word(workspace),
+                                     *dev, (cudaStream_t)stream);
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
 }
 
@@ -178,11 +197,11 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
                          size_t workspace_bytes, void* stream) {
   fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
   if (st != FMLP_OK) return st;
-  if (!x || !gamma || !packed_Wgu || !W_down || !out) return FMLP_ERR_INVALID_ARG;
+  if (!gamma || !packed_Wgu || !W_down) return FMLP_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !out)) return FMLP_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed_Wgu) || !aligned16(W_down) ||
-      !aligned16(out))
+      !aligned16(out) || !aligned16(residual))
     return FMLP_ERR_INVALID_ARG;
-  if (residual && !aligned16(residual)) return FMLP_ERR_INVALID_ARG;
   if (!eps_ok(eps) || !tile_ok(tile_T, I)) return FMLP_ERR_INVALID_ARG;
   if (M == 0) return FMLP_OK;
   const DeviceInfo* dev = nullptr;
@@ -190,9 +209,18 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
   if (st != FMLP_OK) return st;
   const WorkspaceLayout L = workspace_layout(M, d, I);
   void* a = (char*)workspace + L.a;
+  uint32_t* status = status_word(workspace);
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_gateup_gemv(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, *dev, s);
-  if (e == cudaSuccess) e = launch_down_gemv(a, M, W_down, d, I, residual, out, *dev, s);
+  cudaError_t e;
+  if (fused_decode_supported(M, d, I, *dev)) {
+    uint32_t* barrier = (uint32_t*)((char*)workspace + L.barrier);
+    e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, a, residual, out,
+                            status, barrier, *dev, s);
+  } else {
+    e = launch_gateup_stream(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, status, *dev, s);
+    if (e == cudaSuccess)
+      e = launch_down_stream(a, M, W_down, d, I, residual, out, status, *dev, s);
+  }
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
 }
 
@@ -203,7 +231,9 @@ fmlp_status fmlp_device_status(void* workspace, void* stream) {
   cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e == cudaSuccess && word != 0) {
-    e = cudaMemsetAsync(workspace, 0, sizeof(word), s);
+    // a call that gave up may have left the grid-barrier words mid-use:
+    // reset the whole control block along with the status word
+    e = cudaMemsetAsync(workspace, 0, workspace_layout(0, 8, 8).a, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   }
   if (e != cudaSuccess) return cuda_fail(e);

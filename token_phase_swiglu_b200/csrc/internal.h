@@ -18,8 +18,12 @@ struct DeviceInfo {
 cudaError_t current_device_info(const DeviceInfo** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
+// The first 256 bytes are control words: the device status word at 0 and
+// the grid-barrier words of the fused kernel at 64 (count) and 192
+// (generation).
 struct WorkspaceLayout {
-  size_t status = 0;     // uint32 device status word (+ reserved control words)
+  size_t status = 0;     // uint32 device status word
+  size_t barrier = 64;   // uint32 arrival count; generation 128 bytes further on
   size_t a = 0;          // bf16 [M x I] intermediate
   size_t total = 0;
 };
@@ -34,14 +38,30 @@ void note_launches(int n);
 cudaError_t launch_pack(const void* W_gate, const void* W_up, int64_t d, int64_t I, int T,
                         void* packed, cudaStream_t stream);
 
-// a[m, i] = bf16(SiLU(r g) * r u) for all M rows, CUDA-core weight streaming.
-cudaError_t launch_gateup_gemv(const void* x, int64_t M, const void* gamma, float eps,
-                               const void* P, int T, int64_t d, int64_t I, void* a,
-                               const DeviceInfo& dev, cudaStream_t stream);
+// Deadline of every bounded device-side wait (fmlp_set_wait_timeout_ns).
+uint64_t wait_timeout_ns();
+// Testing aid (fmlp_set_fault_injection): nonzero makes every producer
+// withhold its last stage so the consumers' bounded waits expire.
+int fault_injection();
 
-// out[m, n] = sum_i W_down[n, i] a[m, i] (+ residual), CUDA-core weight streaming.
-cudaError_t launch_down_gemv(const void* a, int64_t M, const void* W_down, int64_t d,
-                             int64_t I, const void* residual, float* out,
-                             const DeviceInfo& dev, cudaStream_t stream);
+// a[m, i] = bf16(SiLU(r g) * r u) for all M rows: TMA-bulk weight streaming,
+// CUDA-core dot products.  `status` is the workspace's device status word.
+cudaError_t launch_gateup_stream(const void* x, int64_t M, const void* gamma, float eps,
+                                 const void* P, int T, int64_t d, int64_t I, void* a,
+                                 uint32_t* status, const DeviceInfo& dev, cudaStream_t stream);
+
+// Both steps in one persistent launch with a grid barrier between them; only
+// when all M rows fit one pass (fused_decode_supported).  `barrier` points at
+// the workspace's grid-barrier words.
+bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev);
+cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
+                                const void* P, int T, const void* W_down, int64_t d, int64_t I,
+                                void* a, const void* residual, float* out, uint32_t* status,
+                                uint32_t* barrier, const DeviceInfo& dev, cudaStream_t stream);
+
+// out[m, n] = sum_i W_down[n, i] a[m, i] (+ residual), same streaming scheme.
+cudaError_t launch_down_stream(const void* a, int64_t M, const void* W_down, int64_t d,
+                               int64_t I, const void* residual, float* out, uint32_t* status,
+                               const DeviceInfo& dev, cudaStream_t stream);
 
 }  // namespace fmlp

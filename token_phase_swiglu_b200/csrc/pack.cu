@@ -29,10 +29,13 @@ pack_rows(const uint4* __restrict__ Wg, const uint4* __restrict__ Wu, int64_t dv
 cudaError_t launch_pack(const void* W_gate, const void* W_up, int64_t d, int64_t I, int T,
                         void* packed, cudaStream_t stream) {
   const int64_t rows = 2 * I;
-  const int grid = (int)(rows < 65535 * 4 ? rows : 65535 * 4);
-  pack_rows<<<grid, 256, 0, stream>>>((const uint4*)W_gate, (const uint4*)W_up, d / 8, I, T,
-                                      (uint4*)packed);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows < 65535 * 4 ? rows : 65535 * 4));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  // cudaLaunchKernelEx reports this launch's own error (no stale sticky state)
+  cudaError_t e = cudaLaunchKernelEx(&cfg, pack_rows, (const uint4*)W_gate, (const uint4*)W_up,
+                                     d / 8, I, T, (uint4*)packed);
   if (e == cudaSuccess) note_launches(1);
   return e;
 }
