@@ -142,6 +142,36 @@ FMLP_API fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down
  */
 FMLP_API fmlp_status fmlp_device_status(void* workspace, void* stream);
 
+/*
+ * fmlp_forward_noalloc -- fmlp_forward for callers that cannot allocate
+ * device memory.  The pages have no counterpart; this call exists for code
+ * that is given no allocator, for example a plug-in run by a host engine that
+ * owns all of device memory, or a serving loop that must never call
+ * cudaMalloc/cudaFree because those calls can synchronise the device.
+ *
+ * Instead of a caller workspace it uses one scratch buffer of
+ * FMLP_NOALLOC_SCRATCH_BYTES that the library keeps in every GPU's memory
+ * from the moment the library is loaded until the process exits.  The call
+ * itself allocates nothing.  The first call on a device looks up the
+ * buffer's address for that device (cudaGetSymbolAddress) and caches it;
+ * make that first call before any stream capture.
+ *
+ * Arguments, layouts and precision are those of fmlp_forward, minus the
+ * workspace.  Requests whose workspace (fmlp_workspace_bytes(M, d, I)) would
+ * exceed FMLP_NOALLOC_SCRATCH_BYTES are rejected with FMLP_ERR_UNSUPPORTED
+ * before anything is enqueued.  Each call first clears the buffer's control
+ * words on `stream`, then runs the fmlp_forward kernels on it.  Every call in
+ * the process shares the one buffer: calls that may overlap on the GPU (two
+ * streams, or two threads) race and must not be issued.  A device-side
+ * timeout of such a call is not reported (its outputs are then undefined);
+ * use fmlp_forward with a workspace to read the status word.
+ */
+#define FMLP_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+FMLP_API fmlp_status fmlp_forward_noalloc(const void* x, int64_t M, const void* gamma, float eps,
+                                          const void* packed_Wgu, int tile_T, const void* W_down,
+                                          int64_t d, int64_t I, const void* residual, float* out,
+                                          void* stream);
+
 /* Static, human-readable name of a status code. */
 FMLP_API const char* fmlp_status_string(fmlp_status status);
 

@@ -20,7 +20,7 @@ __all__ = [
     "FMLP_ERR_TIMEOUT", "LIB_PATH", "lib", "fmlp_pack", "fmlp_workspace_bytes", "fmlp_forward",
     "fmlp_gate_up_swiglu", "fmlp_down_proj", "fmlp_device_status", "fmlp_status_string",
     "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "fmlp_set_wait_timeout_ns", "fmlp_set_fault_injection",
-    "EXPORTED_SYMBOLS",
+    "fmlp_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 FMLP_OK, FMLP_ERR_INVALID_ARG, FMLP_ERR_UNSUPPORTED, FMLP_ERR_CUDA, FMLP_ERR_TIMEOUT = range(5)
@@ -42,6 +42,7 @@ _SIGNATURES = {
     "fmlp_kernel_launch_count": (ctypes.c_uint64, []),
     "fmlp_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
     "fmlp_set_fault_injection": (None, [_int]),
+    "fmlp_forward_noalloc": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -145,6 +146,24 @@ def fmlp_forward(x, gamma, eps: float, packed, tile_T: int, W_down, out, workspa
                             d, I, _ptr(residual), _ptr(out), _ptr(workspace),
                             workspace.numel() * workspace.element_size(), _stream(stream)),
            "fmlp_forward")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20   # FMLP_NOALLOC_SCRATCH_BYTES in include/fmlp.h
+
+
+def fmlp_forward_noalloc(x, gamma, eps: float, packed, tile_T: int, W_down, out, residual=None,
+                         stream=None) -> None:
+    """fmlp_forward without a workspace, for callers that cannot allocate device
+    memory (the library's own fixed scratch buffer is used; see include/fmlp.h)."""
+    for t, n in ((x, "x"), (gamma, "gamma"), (packed, "packed"), (W_down, "W_down"),
+                 (residual, "residual")):
+        _bf16(t, n)
+    M, d = x.shape
+    I = W_down.shape[1]
+    _check(lib.fmlp_forward_noalloc(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T,
+                                    _ptr(W_down), d, I, _ptr(residual), _ptr(out),
+                                    _stream(stream)),
+           "fmlp_forward_noalloc")
 
 
 def fmlp_gate_up_swiglu(x, gamma, eps: float, packed, tile_T: int, a, workspace,

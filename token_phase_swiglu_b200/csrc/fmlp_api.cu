@@ -55,6 +55,8 @@ fmlp_status device_for_launch(const DeviceInfo** info) {
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+fmlp_status record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
 uint64_t wait_timeout_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 int fault_injection() { return g_fault.load(std::memory_order_relaxed); }

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "fmlp.h"
+
 namespace fmlp {
 
 // Device attributes, queried once per device and cached (a per-launch
@@ -33,6 +35,9 @@ constexpr uint32_t kStatusTimeout = 1u;
 
 // Count of kernels enqueued by the library (fmlp_kernel_launch_count).
 void note_launches(int n);
+
+// Keep `e` for fmlp_last_cuda_error() and return FMLP_ERR_CUDA.
+fmlp_status record_cuda_error(cudaError_t e);
 
 // ---- kernels ---------------------------------------------------------------
 cudaError_t launch_pack(const void* W_gate, const void* W_up, int64_t d, int64_t I, int T,
