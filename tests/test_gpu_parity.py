@@ -334,7 +334,10 @@ def test_bounded_wait_timeout_reports_and_recovers(fm):
 
 def test_fused_and_two_kernel_paths_agree(fm):
     """For M <= 4 fmlp_forward runs one fused launch; the stage calls run the
-    same phases as two launches.  Same arithmetic, same order: identical bits."""
+    same steps as two launches.  The intermediate a is computed identically;
+    the fused kernel sums the down projection over per-CTA slices of the
+    intermediate dimension in f32 (atomic adds), so the outputs agree to f32
+    summation-order differences."""
     dev = torch.device("cuda:0")
     for (M, d, I) in [(1, 3072, 8192), (3, 1024, 2064), (4, 256, 688)]:
         p = wl.make_problem(M, d, I, seed=21, residual=True)
@@ -351,7 +354,8 @@ def test_fused_and_two_kernel_paths_agree(fm):
         fm.fmlp_down_proj(a, g["W_down"], two, ws, residual=g["residual"])
         torch.cuda.synchronize()
         assert fm.fmlp_device_status(ws) == fm.FMLP_OK
-        assert torch.equal(fused, two)
+        norm, _ = errors(fused.cpu().double().numpy(), two.cpu().double().numpy())
+        assert norm <= 1e-5, norm
 
 
 @pytest.mark.parametrize("M,d,I", [(1, 32768, 64), (4, 32768, 64), (1, 64, 65536), (3, 64, 65536),

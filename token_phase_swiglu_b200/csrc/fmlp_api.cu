@@ -84,14 +84,15 @@ cudaError_t current_device_info(const DeviceInfo** out) {
 }
 
 WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
-  (void)d;
   WorkspaceLayout L;
   size_t off = 0;
   L.status = off;
-  L.barrier = off + 64;
+  L.done = off + 128;
   off += 256;
   L.a = off;
   off += align256((size_t)M * (size_t)I * 2);
+  L.acc = off;
+  off += align256((size_t)(M < 4 ? M : 4) * (size_t)d * 4);
   L.total = off;
   return L;
 }
@@ -215,9 +216,10 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   if (fused_decode_supported(M, d, I, *dev)) {
-    uint32_t* barrier = (uint32_t*)((char*)workspace + L.barrier);
-    e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, a, residual, out,
-                            status, barrier, *dev, s);
+    float* acc = (float*)((char*)workspace + L.acc);
+    uint32_t* done = (uint32_t*)((char*)workspace + L.done);
+    e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out, acc,
+                            done, status, *dev, s);
   } else {
     e = launch_gateup_stream(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, status, *dev, s);
     if (e == cudaSuccess)
@@ -233,7 +235,6 @@ fmlp_status fmlp_device_status(void* workspace, void* stream) {
   cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e == cudaSuccess && word != 0) {
-    // a call that gave up may have left the grid-barrier words mid-use:
     // reset the whole control block along with the status word
     e = cudaMemsetAsync(workspace, 0, workspace_layout(0, 8, 8).a, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -20,13 +20,15 @@ struct DeviceInfo {
 cudaError_t current_device_info(const DeviceInfo** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
-// The first 256 bytes are control words: the device status word at 0 and
-// the grid-barrier words of the fused kernel at 64 (count) and 192
-// (generation).
+// The first 256 bytes are control words: the device status word at 0 and the
+// fused kernel's finished-CTA counter at 128.  Then the bf16 intermediate a
+// [M x I] (two-kernel path) and the fused kernel's f32 accumulator [M x d]
+// (M <= 4); the counter and the accumulator return to zero after every call.
 struct WorkspaceLayout {
   size_t status = 0;     // uint32 device status word
-  size_t barrier = 64;   // uint32 arrival count; generation 128 bytes further on
+  size_t done = 128;     // uint32 finished-CTA counter (fused kernel)
   size_t a = 0;          // bf16 [M x I] intermediate
+  size_t acc = 0;        // f32 [min(M,4) x d] accumulator (fused kernel)
   size_t total = 0;
 };
 WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I);
@@ -55,14 +57,14 @@ cudaError_t launch_gateup_stream(const void* x, int64_t M, const void* gamma, fl
                                  const void* P, int T, int64_t d, int64_t I, void* a,
                                  uint32_t* status, const DeviceInfo& dev, cudaStream_t stream);
 
-// Both steps in one persistent launch with a grid barrier between them; only
-// when all M rows fit one pass (fused_decode_supported).  `barrier` points at
-// the workspace's grid-barrier words.
+// Both steps in one launch, split over the intermediate dimension (M <= 4,
+// fused_decode_supported).  acc / done: the workspace's f32 [M x d]
+// accumulator and finished-CTA counter, zero on entry and on exit.
 bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev);
 cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                                void* a, const void* residual, float* out, uint32_t* status,
-                                uint32_t* barrier, const DeviceInfo& dev, cudaStream_t stream);
+                                const void* residual, float* out, float* acc, uint32_t* done,
+                                uint32_t* status, const DeviceInfo& dev, cudaStream_t stream);
 
 // out[m, n] = sum_i W_down[n, i] a[m, i] (+ residual), same streaming scheme.
 cudaError_t launch_down_stream(const void* a, int64_t M, const void* W_down, int64_t d,

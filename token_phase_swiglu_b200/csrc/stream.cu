@@ -16,11 +16,14 @@
 //   * four consumer warps share every stage: warp w owns gate/up pair w (or
 //     W_down row w) of the group, dots it with the activations held in shared
 //     memory, and arrives on the stage's "empty" mbarrier;
-//   * fused_decode runs both steps in one persistent launch, the "Fusion MLP"
-//     of the pages: the producer streams the W_down rows right behind the
-//     gate/up rows while the consumers finish the gate-up phase, meet at a
-//     grid-wide barrier (every CTA needs all of the intermediate a), and go
-//     on to the down projection, so HBM does not idle between the steps;
+//   * fused_decode runs both steps in one launch, the "Fusion MLP" of the
+//     pages.  CTA b owns a slice of the intermediate dimension: it streams the
+//     gate/up rows of its pairs, keeps its slice of a (rounded to bf16) in
+//     shared memory, then streams the matching column slice of W_down (2-D
+//     TMA tiles of 256 rows) and adds its partial down projection into an f32
+//     accumulator in the workspace (red.global.add).  The last CTA to finish
+//     adds the residual, writes out and re-zeroes the accumulator.  No CTA
+//     waits for another, and `a` never travels through global memory;
 //   * launches use programmatic dependent launch: a kernel's producer starts
 //     streaming weights before the previous kernel on the stream has
 //     finished; only the consumers wait for its results.
@@ -29,44 +32,80 @@
 // and exits.
 #include "common.cuh"
 #include "internal.h"
+#include "tmap.h"
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 #include <set>
 
 namespace fmlp {
 namespace {
 
-constexpr int kConsumers = 4;                     // consumer warps = rows (pairs) per group
+constexpr int kGroup = 4;                         // pairs (gate-up) or rows (down) per group
+constexpr int kConsumers = 2 * kGroup;            // consumer warps: item w & 3, column half w >> 2
 constexpr int kThreads = (kConsumers + 1) * 32;   // warp 0 produces
 constexpr int kMaxStages = 8;
 constexpr int kHeader = 256;                      // full[8], empty[8] mbarriers
 constexpr int64_t kMaxStageBytes = 64 * 1024;
 constexpr uint64_t kDrainNs = 1000000000ull;      // in-flight copies land long before this
-constexpr int kGateRows = 2 * kConsumers;         // rows per gate-up stage (4 gate + 4 up)
-constexpr int kDownRows = kConsumers;             // rows per down stage
+constexpr int kGateRows = 2 * kGroup;             // rows per gate-up stage (4 gate + 4 up)
+constexpr int kDownRows = kGroup;                 // rows per down stage
+constexpr int kBarStage = 1;                      // named barrier: consumer-only sync
+constexpr int kBarGroup = 2;                      // named barrier: per-group combine
 
 static_assert(2 * kMaxStages * 8 <= kHeader, "barrier block overflows its header");
 
 __host__ __device__ constexpr size_t align128(size_t n) { return (n + 127) & ~size_t(127); }
 
-// acc += w . s over 8 elements (w: 8 bf16; s: 8 floats)
-__device__ __forceinline__ float dot8(const uint4& w, const float4& s0, const float4& s1,
-                                      float acc) {
-  acc = fmaf(bf16lo(w.x), s0.x, acc); acc = fmaf(bf16hi(w.x), s0.y, acc);
-  acc = fmaf(bf16lo(w.y), s0.z, acc); acc = fmaf(bf16hi(w.y), s0.w, acc);
-  acc = fmaf(bf16lo(w.z), s1.x, acc); acc = fmaf(bf16hi(w.z), s1.y, acc);
-  acc = fmaf(bf16lo(w.w), s1.z, acc); acc = fmaf(bf16hi(w.w), s1.w, acc);
+// Two f32 lanes in one 64-bit register, for the packed FMA of sm_100.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float hsum2(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
+// bf16 pair (low half = element 2j, high half = element 2j+1) as two f32 lanes
+__device__ __forceinline__ uint64_t bf2(uint32_t w) { return pk2(bf16lo(w), bf16hi(w)); }
+
+// acc += w . s over 8 elements (w: 8 bf16; s: 8 f32), as 4 packed FMAs
+__device__ __forceinline__ uint64_t dot8(const uint4& w, const float4& s0, const float4& s1,
+                                         uint64_t acc) {
+  acc = ffma2(bf2(w.x), pk2(s0.x, s0.y), acc);
+  acc = ffma2(bf2(w.y), pk2(s0.z, s0.w), acc);
+  acc = ffma2(bf2(w.z), pk2(s1.x, s1.y), acc);
+  acc = ffma2(bf2(w.w), pk2(s1.z, s1.w), acc);
   return acc;
 }
 
 // acc += w . v over 8 elements (both bf16)
-__device__ __forceinline__ float dot8bf(const uint4& w, const uint4& v, float acc) {
-  acc = fmaf(bf16lo(w.x), bf16lo(v.x), acc); acc = fmaf(bf16hi(w.x), bf16hi(v.x), acc);
-  acc = fmaf(bf16lo(w.y), bf16lo(v.y), acc); acc = fmaf(bf16hi(w.y), bf16hi(v.y), acc);
-  acc = fmaf(bf16lo(w.z), bf16lo(v.z), acc); acc = fmaf(bf16hi(w.z), bf16hi(v.z), acc);
-  acc = fmaf(bf16lo(w.w), bf16lo(v.w), acc); acc = fmaf(bf16hi(w.w), bf16hi(v.w), acc);
+__device__ __forceinline__ uint64_t dot8bf(const uint4& w, const uint4& v, uint64_t acc) {
+  acc = ffma2(bf2(w.x), bf2(v.x), acc);
+  acc = ffma2(bf2(w.y), bf2(v.y), acc);
+  acc = ffma2(bf2(w.z), bf2(v.z), acc);
+  acc = ffma2(bf2(w.w), bf2(v.w), acc);
   return acc;
+}
+
+// Per-group barrier of all consumer warps; returns true if any of them failed.
+__device__ __forceinline__ bool group_barrier_any(bool failed) {
+  uint32_t any;
+  asm volatile(
+      "{\n .reg .pred q, r;\n setp.ne.u32 q, %1, 0;\n"
+      " bar.red.or.pred r, %2, %3, q;\n selp.u32 %0, 1, 0, r;\n}"
+      : "=r"(any)
+      : "r"((uint32_t)failed), "n"(kBarGroup), "n"(kConsumers * 32)
+      : "memory");
+  return any != 0;
 }
 
 // Packed-row index of gate row i (its up row is T rows further on).
@@ -200,7 +239,7 @@ struct GateUpGeom {
 
 __device__ bool produce_gateup(Producer& pr, const GateUpGeom& g, int g0, int n_groups) {
   for (int j = 0; j < n_groups; ++j) {
-    const __nv_bfloat16* pg = g.P + gate_row((g0 + j) * kConsumers, g.T) * g.d;
+    const __nv_bfloat16* pg = g.P + gate_row((g0 + j) * kGroup, g.T) * g.d;
     const __nv_bfloat16* pu = pg + (int64_t)g.T * g.d;
     for (int ch = 0; ch < g.nchunks; ++ch) {
       if (!pr.acquire()) return false;
@@ -212,13 +251,13 @@ __device__ bool produce_gateup(Producer& pr, const GateUpGeom& g, int g0, int n_
       mbar_arrive_expect_tx(bar, (uint32_t)(kGateRows * len * 2));
       if (g.nchunks == 1) {
         // 4 whole gate rows, then the 4 whole up rows: two contiguous runs
-        const uint32_t run = (uint32_t)(kConsumers * g.d * 2);
+        const uint32_t run = (uint32_t)(kGroup * g.d * 2);
         bulk_copy_g2s(buf, pg, run, bar, pr.pol);
         bulk_copy_g2s(buf + run, pu, run, bar, pr.pol);
       } else {
         for (int r = 0; r < kGateRows; ++r) {
           const __nv_bfloat16* row =
-              r < kConsumers ? pg + (int64_t)r * g.d : pu + (int64_t)(r - kConsumers) * g.d;
+              r < kGroup ? pg + (int64_t)r * g.d : pu + (int64_t)(r - kGroup) * g.d;
           bulk_copy_g2s(buf + (size_t)r * g.kc * 2, row + k0, (uint32_t)len * 2u, bar, pr.pol);
         }
       }
@@ -229,6 +268,7 @@ __device__ bool produce_gateup(Producer& pr, const GateUpGeom& g, int g0, int n_
 }
 
 // s = x * gamma (exact in f32) for the CTA's token rows, and r = 1/sqrt(mean x^2 + eps).
+// Row m of s holds d/8 float4 of columns 8v..8v+3, then d/8 float4 of 8v+4..8v+7.
 template <int MT>
 __device__ void stage_x_gamma(const __nv_bfloat16* x, const __nv_bfloat16* gamma, float eps,
                               int d, int m0, int mt, float* s, float (*red)[MT], float* rinv) {
@@ -248,9 +288,11 @@ __device__ void stage_x_gamma(const __nv_bfloat16* x, const __nv_bfloat16* gamma
                            bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
 #pragma unroll
       for (int e = 0; e < 8; ++e) ss[m] = fmaf(xf[e], xf[e], ss[m]);
-      float4* dst = reinterpret_cast<float4*>(s + (int64_t)m * d + (int64_t)v * 8);
-      dst[0] = make_float4(xf[0] * gf[0], xf[1] * gf[1], xf[2] * gf[2], xf[3] * gf[3]);
-      dst[1] = make_float4(xf[4] * gf[4], xf[5] * gf[5], xf[6] * gf[6], xf[7] * gf[7]);
+      // two planes of float4 (columns 8v..8v+3, then 8v+4..8v+7) so that lanes
+      // reading consecutive vectors touch consecutive 16-byte words
+      float4* dst = reinterpret_cast<float4*>(s + (int64_t)m * d);
+      dst[v] = make_float4(xf[0] * gf[0], xf[1] * gf[1], xf[2] * gf[2], xf[3] * gf[3]);
+      dst[d / 8 + v] = make_float4(xf[4] * gf[4], xf[5] * gf[5], xf[6] * gf[6], xf[7] * gf[7]);
     }
   }
 #pragma unroll
@@ -258,7 +300,7 @@ __device__ void stage_x_gamma(const __nv_bfloat16* x, const __nv_bfloat16* gamma
     const float t = warp_sum(ss[m]);
     if (lane == 0) red[c][m] = t;
   }
-  named_barrier_sync(1, kConsumers * 32);
+  named_barrier_sync(kBarStage, kConsumers * 32);
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     float t = 0.f;
@@ -268,61 +310,79 @@ __device__ void stage_x_gamma(const __nv_bfloat16* x, const __nv_bfloat16* gamma
   }
 }
 
-// Consumer warp c: pair c of every group; writes a[m, i] for its pairs.
+// Consumer warps: pair w & 3 of every group, column half w >> 2; writes a[m, i].
+// xch: [2][kGroup][2*MT] floats of shared memory for the halves' partial sums.
+// If `slice` is given, a goes to shared memory instead: slice[m * slice_ld +
+// (i - slice_i0)] holds the bf16-rounded value as f32.
 template <int MT>
 __device__ bool consume_gateup(Consumer& cs, const GateUpGeom& g, int g0, int n_groups,
                                const float* s, const float* rinv, __nv_bfloat16* a, int m0,
-                               int mt) {
+                               int mt, float* xch, float* slice = nullptr, int slice_i0 = 0,
+                               int slice_ld = 0) {
   const int c = (threadIdx.x >> 5) - 1, lane = cs.lane;
+  const int pr = c & (kGroup - 1), half = c / kGroup;
   for (int j = 0; j < n_groups; ++j) {
-    float ag[2][MT], au[2][MT];
+    uint64_t ag[2][MT], au[2][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) ag[0][m] = ag[1][m] = au[0][m] = au[1][m] = 0.f;
-    for (int ch = 0; ch < g.nchunks; ++ch) {
+    for (int m = 0; m < MT; ++m) ag[0][m] = ag[1][m] = au[0][m] = au[1][m] = 0ull;
+    bool ok = true;
+    for (int ch = 0; ch < g.nchunks && ok; ++ch) {
       const uint8_t* buf = cs.wait_full();
-      if (!buf) return false;
+      if (!buf) {
+        ok = false;
+        break;
+      }
       const int k0 = ch * g.kc;
       const int nv = min(g.kc, g.d - k0) / 8;
-      const uint8_t* bg = buf + (size_t)c * g.kc * 2;
-      const uint8_t* bu = buf + (size_t)(kConsumers + c) * g.kc * 2;
-      const float* sk = s + k0;
-      int v = lane;
-      for (; v + 32 < nv; v += 64) {  // two independent accumulator sets
+      const uint8_t* bg = buf + (size_t)pr * g.kc * 2;
+      const uint8_t* bu = buf + (size_t)(kGroup + pr) * g.kc * 2;
+      const int kv0 = k0 / 8;
+      for (int v = lane + 32 * half; v < nv; v += 128) {  // vectors v and v + 64
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int vv = v + 32 * h;
-          const uint4 wg = lds128(bg + 16 * vv);
-          const uint4 wu = lds128(bu + 16 * vv);
+          const int vv = v + 64 * h;
+          if (h == 0 || vv < nv) {
+            const uint4 wg = lds128(bg + 16 * vv);
+            const uint4 wu = lds128(bu + 16 * vv);
 #pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            const float4* sp = reinterpret_cast<const float4*>(sk + (int64_t)m * g.d + 8 * vv);
-            const float4 s0 = sp[0], s1 = sp[1];
-            ag[h][m] = dot8(wg, s0, s1, ag[h][m]);
-            au[h][m] = dot8(wu, s0, s1, au[h][m]);
+            for (int m = 0; m < MT; ++m) {
+              const float4* sp = reinterpret_cast<const float4*>(s + (int64_t)m * g.d) + kv0 + vv;
+              const float4 s0 = sp[0], s1 = sp[g.d / 8];
+              ag[h][m] = dot8(wg, s0, s1, ag[h][m]);
+              au[h][m] = dot8(wu, s0, s1, au[h][m]);
+            }
           }
-        }
-      }
-      if (v < nv) {
-        const uint4 wg = lds128(bg + 16 * v);
-        const uint4 wu = lds128(bu + 16 * v);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          const float4* sp = reinterpret_cast<const float4*>(sk + (int64_t)m * g.d + 8 * v);
-          const float4 s0 = sp[0], s1 = sp[1];
-          ag[0][m] = dot8(wg, s0, s1, ag[0][m]);
-          au[0][m] = dot8(wu, s0, s1, au[0][m]);
         }
       }
       cs.release();
     }
-    const int item = (g0 + j) * kConsumers + c;
+    float gs[MT], us[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      const float gs = warp_sum(ag[0][m] + ag[1][m]);
-      const float us = warp_sum(au[0][m] + au[1][m]);
-      if (lane == m && m < mt)
-        a[(int64_t)(m0 + m) * g.I + item] =
-            __float2bfloat16_rn(silu_mul(gs * rinv[m], us * rinv[m]));
+      gs[m] = warp_sum(hsum2(ag[0][m]) + hsum2(ag[1][m]));
+      us[m] = warp_sum(hsum2(au[0][m]) + hsum2(au[1][m]));
+    }
+    float* x2 = xch + ((j & 1) * kGroup + pr) * 2 * MT;
+    if (half == 1 && lane == 0) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        x2[m] = gs[m];
+        x2[MT + m] = us[m];
+      }
+    }
+    if (group_barrier_any(!ok)) return false;
+    if (half == 0) {
+      const int item = (g0 + j) * kGroup + pr;
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (lane == m) {
+          const float gt = gs[m] + x2[m], ut = us[m] + x2[MT + m];
+          const __nv_bfloat16 av = __float2bfloat16_rn(silu_mul(gt * rinv[m], ut * rinv[m]));
+          if (slice)
+            slice[m * slice_ld + (item - slice_i0)] = m < mt ? __bfloat162float(av) : 0.f;
+          else if (m < mt)
+            a[(int64_t)(m0 + m) * g.I + item] = av;
+        }
     }
   }
   return true;
@@ -373,77 +433,65 @@ __device__ void stage_a(const __nv_bfloat16* a, int I, int m0, int mt, uint8_t* 
       if (m < mt) av = ld_keep(a + (int64_t)(m0 + m) * I + (int64_t)v * 8);
       *reinterpret_cast<uint4*>(act + ((size_t)m * I + (size_t)v * 8) * 2) = av;
     }
-  named_barrier_sync(1, kConsumers * 32);
+  named_barrier_sync(kBarStage, kConsumers * 32);
 }
 
+// Consumer warps: row w & 3 of every group, column half w >> 2.
 template <int MT>
 __device__ bool consume_down(Consumer& cs, const DownGeom& g, int g0, int n_groups,
                              const uint8_t* act, const __nv_bfloat16* residual, float* out,
-                             int m0, int mt) {
+                             int m0, int mt, float* xch) {
   const int c = (threadIdx.x >> 5) - 1, lane = cs.lane;
+  const int row = c & (kGroup - 1), half = c / kGroup;
   for (int j = 0; j < n_groups; ++j) {
-    float acc[2][MT];
+    uint64_t acc[2][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[0][m] = acc[1][m] = 0.f;
-    for (int ch = 0; ch < g.nchunks; ++ch) {
+    for (int m = 0; m < MT; ++m) acc[0][m] = acc[1][m] = 0ull;
+    bool ok = true;
+    for (int ch = 0; ch < g.nchunks && ok; ++ch) {
       const uint8_t* buf = cs.wait_full();
-      if (!buf) return false;
+      if (!buf) {
+        ok = false;
+        break;
+      }
       const int k0 = ch * g.kc;
       const int nv = min(g.kc, g.I - k0) / 8;
-      const uint8_t* bw = buf + (size_t)c * g.kc * 2;
+      const uint8_t* bw = buf + (size_t)row * g.kc * 2;
       const uint8_t* ak = act + (size_t)k0 * 2;
-      int v = lane;
-      for (; v + 32 < nv; v += 64) {
+      for (int v = lane + 32 * half; v < nv; v += 128) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int vv = v + 32 * h;
-          const uint4 w = lds128(bw + 16 * vv);
+          const int vv = v + 64 * h;
+          if (h == 0 || vv < nv) {
+            const uint4 w = lds128(bw + 16 * vv);
 #pragma unroll
-          for (int m = 0; m < MT; ++m)
-            acc[h][m] = dot8bf(w, lds128(ak + ((size_t)m * g.I + 8 * vv) * 2), acc[h][m]);
+            for (int m = 0; m < MT; ++m)
+              acc[h][m] = dot8bf(w, lds128(ak + ((size_t)m * g.I + 8 * vv) * 2), acc[h][m]);
+          }
         }
-      }
-      if (v < nv) {
-        const uint4 w = lds128(bw + 16 * v);
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-          acc[0][m] = dot8bf(w, lds128(ak + ((size_t)m * g.I + 8 * v) * 2), acc[0][m]);
       }
       cs.release();
     }
-    const int n = (g0 + j) * kDownRows + c;
+    float t[MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      const float t = warp_sum(acc[0][m] + acc[1][m]);
-      if (lane == m && m < mt) {
-        float o = t;
-        if (residual) o += __bfloat162float(residual[(int64_t)(m0 + m) * g.d + n]);
-        out[(int64_t)(m0 + m) * g.d + n] = o;
-      }
+    for (int m = 0; m < MT; ++m) t[m] = warp_sum(hsum2(acc[0][m]) + hsum2(acc[1][m]));
+    float* x2 = xch + ((j & 1) * kGroup + row) * 2 * MT;
+    if (half == 1 && lane == 0) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m) x2[m] = t[m];
+    }
+    if (group_barrier_any(!ok)) return false;
+    if (half == 0) {
+      const int n = (g0 + j) * kDownRows + row;
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (lane == m && m < mt) {
+          float o = t[m] + x2[m];
+          if (residual) o += __bfloat162float(residual[(int64_t)(m0 + m) * g.d + n]);
+          out[(int64_t)(m0 + m) * g.d + n] = o;
+        }
     }
   }
-  return true;
-}
-
-// Grid-wide barrier between the two phases of fused_decode, run by one thread
-// per CTA.  `count` returns to zero after every use; `gen` is a free-running
-// generation counter.  Bounded: gives up after wait_ns.
-__device__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t nblocks,
-                             uint64_t wait_ns) {
-  const uint32_t g = ld_acquire_gpu(gen);
-  __threadfence();
-  if (atomicAdd(count, 1u) == nblocks - 1) {
-    atomicExch(count, 0u);
-    __threadfence();
-    atomicAdd(gen, 1u);
-    return true;
-  }
-  const uint64_t t0 = globaltimer_ns();
-  while (ld_acquire_gpu(gen) == g) {
-    __nanosleep(64);
-    if (globaltimer_ns() - t0 > wait_ns) return false;
-  }
-  __threadfence();
   return true;
 }
 
@@ -456,7 +504,6 @@ struct StreamParams {
   const __nv_bfloat16* residual;
   __nv_bfloat16* a;      // intermediate (output of the gate-up phase)
   float* out;
-  uint32_t* barrier;     // fused: [0] arrival count, [32] generation (separate lines)
   Control ctl;
   GateUpGeom gu;
   DownGeom dn;
@@ -469,6 +516,7 @@ template <int MT, bool GATE, bool DOWN>
 __device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_bytes) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ float red[kConsumers][MT];
+  __shared__ float xch[2 * kGroup * 2 * MT];
   __shared__ CtaState st;
 
   Ring ring;
@@ -483,8 +531,8 @@ __device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_by
   const int m0 = blockIdx.y * MT;
   const int mt = min(MT, p.M - m0);
   int ga0 = 0, nga = 0, gd0 = 0, ngd = 0;
-  if (GATE) split_groups(p.gu.I / kConsumers, blockIdx.x, gridDim.x, false, ga0, nga);
-  if (DOWN) split_groups(p.dn.d / kDownRows, blockIdx.x, gridDim.x, GATE, gd0, ngd);
+  if (GATE) split_groups(p.gu.I / kGroup, blockIdx.x, gridDim.x, false, ga0, nga);
+  if (DOWN) split_groups(p.dn.d / kDownRows, blockIdx.x, gridDim.x, false, gd0, ngd);
 
   if (threadIdx.x == 0) init_ring(ring, st);
   __syncthreads();
@@ -499,6 +547,7 @@ __device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_by
       if (DOWN && ok) produce_down(pr, p.dn, gd0, ngd);
       st.issued = pr.k;
     }
+    __syncwarp();
   } else {
     grid_dependency_wait();  // inputs may be written by the previous kernel
     Consumer cs{ring, &st, p.ctl, 0, lane};
@@ -508,20 +557,11 @@ __device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_by
       stage_x_gamma<MT>(p.x, p.gamma, p.eps, p.gu.d, m0, mt, reinterpret_cast<float*>(act),
                         red, rinv);
       ok = consume_gateup<MT>(cs, p.gu, ga0, nga, reinterpret_cast<const float*>(act), rinv,
-                              p.a, m0, mt);
-    }
-    if (GATE && DOWN) {
-      // every CTA needs all of a: grid-wide barrier (act is then reused for a)
-      named_barrier_sync(1, kConsumers * 32);
-      if (threadIdx.x == 32 && !grid_barrier(p.barrier, p.barrier + 32, gridDim.x,
-                                             p.ctl.wait_ns))
-        flag_timeout(&st, p.ctl.status);
-      named_barrier_sync(1, kConsumers * 32);
-      ok = ok && !st.abort;
+                              p.a, m0, mt, xch);
     }
     if (DOWN && ok) {
       stage_a<MT>(p.a, p.dn.I, m0, mt, act);
-      consume_down<MT>(cs, p.dn, gd0, ngd, act, p.residual, p.out, m0, mt);
+      consume_down<MT>(cs, p.dn, gd0, ngd, act, p.residual, p.out, m0, mt, xch);
     }
   }
   __syncthreads();
@@ -538,11 +578,190 @@ __global__ void __launch_bounds__(kThreads, 1) down_stream(const StreamParams p)
   stream_body<MT, false, true>(p, align128((size_t)MT * p.dn.I * 2));
 }
 
+// ---------------------------------------------------------------------------
+// fused_decode: both steps in one launch, split over the intermediate dimension.
+// ---------------------------------------------------------------------------
+struct FusedParams {
+  CUtensorMap wd_map;  // W_down [d x I] bf16, boxes of rows_d x swbox, no swizzle
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* gamma;
+  const __nv_bfloat16* residual;
+  float* out;
+  float* acc;          // [M x d] f32 accumulator (zero between calls)
+  uint32_t* done;      // CTAs finished (zero between calls)
+  Control ctl;
+  GateUpGeom gu;
+  float eps;
+  int M, d, I;
+  int units;           // I / 8: slices are cut at multiples of 8 pairs (16-byte columns)
+  int swbox;           // W_down slice box width (>= every CTA's slice, odd multiple of 8)
+  int rows_d;          // W_down rows per stage (256, or 128 for wide slices)
+  int nrb;             // row blocks = ceil(d / rows_d)
+  int stages, stage_bytes;
+};
+
+__device__ void produce_down_slice(Producer& pr, const FusedParams& p, int i0) {
+  const uint32_t bytes = (uint32_t)(p.swbox * p.rows_d * 2);
+  for (int rb = 0; rb < p.nrb; ++rb) {
+    if (!pr.acquire()) return;
+    const int slot = pr.k % pr.ring.stages;
+    uint64_t* bar = &pr.ring.full[slot];
+    mbar_arrive_expect_tx(bar, bytes);  // a box always lands whole (zeros past the edges)
+    tma_load_2d(pr.ring.buf(slot), &p.wd_map, i0, rb * p.rows_d, bar, pr.pol);
+    ++pr.k;
+  }
+}
+
+// Each consumer thread owns one W_down row of the stage (two threads per row,
+// column halves, when rows_d == 128) and adds its partial dot products with
+// the CTA's slice of a into acc.
 template <int MT>
-__global__ void __launch_bounds__(kThreads, 1) fused_decode(const StreamParams p) {
-  const size_t act_g = align128((size_t)MT * p.gu.d * sizeof(float));
-  const size_t act_d = align128((size_t)MT * p.dn.I * 2);
-  stream_body<MT, true, true>(p, act_g > act_d ? act_g : act_d);
+__device__ bool consume_down_slice(Consumer& cs, const FusedParams& p, const float* slice,
+                                   int w, int mt) {
+  const int ct = threadIdx.x - 32;
+  const int r = p.rows_d == 256 ? ct : (ct & 127);
+  int c0 = 0, c1 = w;
+  if (p.rows_d != 256) {
+    const int hw = ((w / 2) + 7) / 8 * 8;
+    if (ct < 128) c1 = hw; else c0 = hw;
+  }
+  for (int rb = 0; rb < p.nrb; ++rb) {
+    const uint8_t* buf = cs.wait_full();
+    if (!buf) return false;
+    const int n = rb * p.rows_d + r;
+    if (n < p.d) {
+      const uint8_t* row = buf + (size_t)r * p.swbox * 2;
+      float acc[2][MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[0][m] = acc[1][m] = 0.f;
+      int c = c0;
+      for (; c + 8 < c1; c += 16) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 wv = lds128(row + 2 * (c + 8 * h));
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float4* ap = reinterpret_cast<const float4*>(slice + m * p.swbox + c + 8 * h);
+            const float4 a0 = ap[0], a1 = ap[1];
+            float t = acc[h][m];
+            t = fmaf(bf16lo(wv.x), a0.x, t); t = fmaf(bf16hi(wv.x), a0.y, t);
+            t = fmaf(bf16lo(wv.y), a0.z, t); t = fmaf(bf16hi(wv.y), a0.w, t);
+            t = fmaf(bf16lo(wv.z), a1.x, t); t = fmaf(bf16hi(wv.z), a1.y, t);
+            t = fmaf(bf16lo(wv.w), a1.z, t); t = fmaf(bf16hi(wv.w), a1.w, t);
+            acc[h][m] = t;
+          }
+        }
+      }
+      if (c < c1) {
+        const uint4 wv = lds128(row + 2 * c);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float4* ap = reinterpret_cast<const float4*>(slice + m * p.swbox + c);
+          const float4 a0 = ap[0], a1 = ap[1];
+          float t = acc[0][m];
+          t = fmaf(bf16lo(wv.x), a0.x, t); t = fmaf(bf16hi(wv.x), a0.y, t);
+          t = fmaf(bf16lo(wv.y), a0.z, t); t = fmaf(bf16hi(wv.y), a0.w, t);
+          t = fmaf(bf16lo(wv.z), a1.x, t); t = fmaf(bf16hi(wv.z), a1.y, t);
+          t = fmaf(bf16lo(wv.w), a1.z, t); t = fmaf(bf16hi(wv.w), a1.w, t);
+          acc[0][m] = t;
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (m < mt) atomicAdd(p.acc + (int64_t)m * p.d + n, acc[0][m] + acc[1][m]);
+    }
+    cs.release();
+  }
+  return true;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constant__ FusedParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ float red[kConsumers][MT];
+  __shared__ float xch[2 * kGroup * 2 * MT];
+  __shared__ CtaState st;
+  __shared__ int last_cta;
+
+  Ring ring;
+  ring.full = reinterpret_cast<uint64_t*>(smem);
+  ring.empty = ring.full + kMaxStages;
+  float* s = reinterpret_cast<float*>(smem + kHeader);                          // [MT][d]
+  float* slice = reinterpret_cast<float*>(smem + kHeader + align128((size_t)MT * p.d * 4));
+  ring.stage0 = smem + kHeader + align128((size_t)MT * p.d * 4) +
+                align128((size_t)MT * p.swbox * 4);
+  ring.stages = p.stages;
+  ring.stage_bytes = p.stage_bytes;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = min(MT, p.M);
+  int u0, nu;
+  split_groups(p.units, blockIdx.x, gridDim.x, false, u0, nu);
+  const int i0 = u0 * 8, w = nu * 8;
+  const int g0 = i0 / kGroup, ng = w / kGroup;
+
+  if (threadIdx.x == 0) init_ring(ring, st);
+  __syncthreads();
+  grid_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      Producer pr{ring, &st, p.ctl, evict_first_policy(), ng * p.gu.nchunks + p.nrb};
+      if (produce_gateup(pr, p.gu, g0, ng)) produce_down_slice(pr, p, i0);
+      st.issued = pr.k;
+    }
+    __syncwarp();
+  } else {
+    grid_dependency_wait();  // inputs may be written by the previous kernel
+    const int ct = threadIdx.x - 32;
+    Consumer cs{ring, &st, p.ctl, 0, lane};
+    float rinv[MT];
+    stage_x_gamma<MT>(p.x, p.gamma, p.eps, p.d, 0, mt, s, red, rinv);
+    bool ok = consume_gateup<MT>(cs, p.gu, g0, ng, s, rinv, nullptr, 0, mt, xch, slice, i0,
+                                 p.swbox);
+    named_barrier_sync(kBarStage, kConsumers * 32);  // the CTA's slice of a is complete
+    if (ok) consume_down_slice<MT>(cs, p, slice, w, mt);
+    // Completion count, also after a timeout, so that the last CTA always
+    // leaves acc and the counter at zero for the next call.
+    __threadfence();
+    named_barrier_sync(kBarStage, kConsumers * 32);
+    if (ct == 0) last_cta = atomicAdd(p.done, 1u) == gridDim.x - 1;
+    named_barrier_sync(kBarStage, kConsumers * 32);
+    if (last_cta) {
+      // out = acc (+ residual); acc back to zero.  d % 8 == 0, so float4 and
+      // four-element residual reads tile every row; all loads are issued
+      // before the stores to pay the L2 latency once.
+      __threadfence();
+      constexpr int kBatch = 8;
+      const int n4 = mt * p.d / 4;
+      for (int base = ct; base < n4; base += kConsumers * 32 * kBatch) {
+        float4 v[kBatch];
+        uint2 r[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          const int i = base + b * kConsumers * 32;
+          if (i < n4) {
+            v[b] = __ldcg(reinterpret_cast<const float4*>(p.acc) + i);
+            r[b] = p.residual ? __ldg(reinterpret_cast<const uint2*>(p.residual) + i)
+                              : make_uint2(0, 0);
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          const int i = base + b * kConsumers * 32;
+          if (i < n4) {
+            __stcg(reinterpret_cast<float4*>(p.acc) + i, make_float4(0.f, 0.f, 0.f, 0.f));
+            reinterpret_cast<float4*>(p.out)[i] =
+                make_float4(v[b].x + bf16lo(r[b].x), v[b].y + bf16hi(r[b].x),
+                            v[b].z + bf16lo(r[b].y), v[b].w + bf16hi(r[b].y));
+          }
+        }
+      }
+      if (ct == 0) atomicExch(p.done, 0u);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && st.abort) drain_ring(ring, st.issued);
 }
 
 // ---------------------------------------------------------------------------
@@ -637,15 +856,13 @@ Plan make_plan(int64_t M, int64_t d, int64_t I, bool gate, bool down, const Devi
 
 StreamParams make_params(const Plan& pl, const void* x, int64_t M, const void* gamma, float eps,
                          const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                         void* a, const void* residual, float* out, uint32_t* status,
-                         uint32_t* barrier) {
+                         void* a, const void* residual, float* out, uint32_t* status) {
   StreamParams p = {};
   p.x = (const __nv_bfloat16*)x;
   p.gamma = (const __nv_bfloat16*)gamma;
   p.residual = (const __nv_bfloat16*)residual;
   p.a = (__nv_bfloat16*)a;
   p.out = out;
-  p.barrier = barrier;
   p.ctl.status = status;
   p.ctl.wait_ns = wait_timeout_ns();
   p.ctl.drop_last = fault_injection();
@@ -665,7 +882,6 @@ StreamParams make_params(const Plan& pl, const void* x, int64_t M, const void* g
   };
 FMLP_KERNEL_TAG(gateup_stream)
 FMLP_KERNEL_TAG(down_stream)
-FMLP_KERNEL_TAG(fused_decode)
 #undef FMLP_KERNEL_TAG
 
 template <template <int> class Tag>
@@ -687,8 +903,8 @@ cudaError_t launch_gateup_stream(const void* x, int64_t M, const void* gamma, fl
   const Plan pl = make_plan(M, d, I, true, false, dev);
   if (pl.mt == 0) return cudaErrorInvalidConfiguration;
   const StreamParams p = make_params(pl, x, M, gamma, eps, P, T, nullptr, d, I, a, nullptr,
-                                     nullptr, status, nullptr);
-  const dim3 grid((unsigned)std::min<int64_t>(I / kConsumers, dev.sm_count),
+                                     nullptr, status);
+  const dim3 grid((unsigned)std::min<int64_t>(I / kGroup, dev.sm_count),
                   (unsigned)((M + pl.mt - 1) / pl.mt));
   return launch_mt<gateup_stream_tag>(pl.mt, grid, pl, dev, stream, p);
 }
@@ -699,29 +915,117 @@ cudaError_t launch_down_stream(const void* a, int64_t M, const void* W_down, int
   const Plan pl = make_plan(M, d, I, false, true, dev);
   if (pl.mt == 0) return cudaErrorInvalidConfiguration;
   const StreamParams p = make_params(pl, nullptr, M, nullptr, 0.f, nullptr, 0, W_down, d, I,
-                                     const_cast<void*>(a), residual, out, status, nullptr);
+                                     const_cast<void*>(a), residual, out, status);
   const dim3 grid((unsigned)std::min<int64_t>(d / kDownRows, dev.sm_count),
                   (unsigned)((M + pl.mt - 1) / pl.mt));
   return launch_mt<down_stream_tag>(pl.mt, grid, pl, dev, stream, p);
 }
 
+namespace {
+
+struct FusedPlan {
+  int mt = 0, grid = 0, units = 0, swbox = 0, rows_d = 0, nrb = 0, stages = 0, stage_bytes = 0;
+  Chunking gu;
+  size_t smem = 0;
+};
+
+// One pass over the weights (all M <= 4 rows per CTA), a slice of at most
+// 256 columns per CTA, and a ring of at least three stages.
+FusedPlan make_fused_plan(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev) {
+  FusedPlan f;
+  if (M < 1 || M > 4) return f;
+  const size_t budget = (size_t)dev.max_smem_optin - 1024;
+  f.units = (int)(I / 8);
+  f.grid = std::min(f.units, dev.sm_count);
+  const int max_units = (f.units + f.grid - 1) / f.grid;
+  int sw_units = max_units | 1;  // odd count of 16-byte columns: conflict-free row reads
+  f.swbox = 8 * sw_units;
+  if (f.swbox > 256) return FusedPlan();
+  f.rows_d = f.swbox <= 128 ? 256 : 128;
+  f.nrb = (int)((d + f.rows_d - 1) / f.rows_d);
+  const size_t down_stage = align128((size_t)f.swbox * f.rows_d * 2);
+  const size_t act = align128((size_t)M * d * 4) + align128((size_t)M * f.swbox * 4);
+  if (kHeader + act >= budget) return FusedPlan();
+  for (int64_t target = kMaxStageBytes; target >= 4096; target /= 2) {
+    const Chunking gu = chunk_rows(d, kGateRows, target);
+    const size_t slot = std::max<size_t>(gu.stage_bytes, down_stage);
+    const size_t fit = (budget - kHeader - act) / slot;
+    if (fit < 3) continue;
+    f.gu = gu;
+    f.mt = (int)M;
+    f.stage_bytes = (int)slot;
+    f.stages = (int)std::min<size_t>(kMaxStages, fit);
+    f.smem = kHeader + act + (size_t)f.stages * slot;
+    return f;
+  }
+  return FusedPlan();
+}
+
+template <int MT>
+cudaError_t launch_fused_mt(const FusedPlan& f, const DeviceInfo& dev, cudaStream_t stream,
+                            const FusedParams& p) {
+  auto kernel = fused_decode<MT>;
+  cudaError_t e = allow_max_smem(kernel, dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)f.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = f.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kernel, p);
+  if (e == cudaSuccess) note_launches(1);
+  return e;
+}
+
+}  // namespace
+
 bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev) {
-  const Plan pl = make_plan(M, d, I, true, true, dev);
-  return pl.mt != 0 && pl.mt >= M;  // one pass over the weights: all rows in one CTA row
+  return make_fused_plan(M, d, I, dev).mt != 0;
 }
 
 cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                                void* a, const void* residual, float* out, uint32_t* status,
-                                uint32_t* barrier, const DeviceInfo& dev, cudaStream_t stream) {
-  const Plan pl = make_plan(M, d, I, true, true, dev);
-  if (pl.mt == 0 || pl.mt < M) return cudaErrorInvalidConfiguration;
-  const StreamParams p = make_params(pl, x, M, gamma, eps, P, T, W_down, d, I, a, residual, out,
-                                     status, barrier);
-  // one CTA per SM at most, so every CTA is resident for the grid barrier
-  const int groups = (int)std::min<int64_t>(I / kConsumers, d / kDownRows);
-  const dim3 grid((unsigned)std::min(groups, dev.sm_count), 1);
-  return launch_mt<fused_decode_tag>(pl.mt, grid, pl, dev, stream, p);
+                                const void* residual, float* out, float* acc, uint32_t* done,
+                                uint32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
+  const FusedPlan f = make_fused_plan(M, d, I, dev);
+  if (f.mt == 0) return cudaErrorInvalidConfiguration;
+  FusedParams p;
+  memset(&p, 0, sizeof(p));
+  cudaError_t e = encode_tmap_2d_bf16(&p.wd_map, W_down, (uint64_t)d, (uint64_t)I,
+                                      (uint64_t)I * 2, (uint32_t)f.rows_d, (uint32_t)f.swbox,
+                                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (e != cudaSuccess) return e;
+  p.x = (const __nv_bfloat16*)x;
+  p.gamma = (const __nv_bfloat16*)gamma;
+  p.residual = (const __nv_bfloat16*)residual;
+  p.out = out;
+  p.acc = acc;
+  p.done = done;
+  p.ctl.status = status;
+  p.ctl.wait_ns = wait_timeout_ns();
+  p.ctl.drop_last = fault_injection();
+  p.gu = GateUpGeom{(const __nv_bfloat16*)P, T, (int)d, (int)I, f.gu.kc, f.gu.nchunks};
+  p.eps = eps;
+  p.M = (int)M;
+  p.d = (int)d;
+  p.I = (int)I;
+  p.units = f.units;
+  p.swbox = f.swbox;
+  p.rows_d = f.rows_d;
+  p.nrb = f.nrb;
+  p.stages = f.stages;
+  p.stage_bytes = f.stage_bytes;
+  switch (f.mt) {
+    case 1: return launch_fused_mt<1>(f, dev, stream, p);
+    case 2: return launch_fused_mt<2>(f, dev, stream, p);
+    case 3: return launch_fused_mt<3>(f, dev, stream, p);
+    default: return launch_fused_mt<4>(f, dev, stream, p);
+  }
 }
 
 }  // namespace fmlp

@@ -1,0 +1,17 @@
+// TMA tensor-map encoding (driver entry point looked up once through the runtime).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fmlp {
+
+// 2-D bf16 tensor map over a row-major matrix of `rows` x `cols` elements
+// (row stride `row_bytes`), copying boxes of box_rows x box_cols with no
+// swizzle (or the given swizzle); out-of-range elements read as zero.
+cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                                uint64_t row_bytes, uint32_t box_rows, uint32_t box_cols,
+                                CUtensorMapSwizzle swizzle);
+
+}  // namespace fmlp
