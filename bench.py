@@ -41,6 +41,7 @@ EPS = 1e-5
 TILE_T = 16
 METRIC = "fused-MLP weight-stream GB/s (% B200 HBM peak) and tokens/s per layer at 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 # ----------------------------------------------------------------------------
@@ -424,11 +425,22 @@ def run_ours(args) -> None:
     else:
         peak, peak_src = FALLBACK_HBM_GBS, "fallback"
     fused = per_step is not None and per_step == L   # one kernel per layer
+    if "bf16_tflops" in peaks:
+        tpeak, tpeak_src = float(peaks["bf16_tflops"]), "measured"
+    else:
+        tpeak, tpeak_src = FALLBACK_BF16_TFLOPS, "fallback"
+    gu_flops = 4 * M * d * I                      # algorithmic gate-up FLOPs
     if fused:
         kname, kbytes, kms = "fused_decode", algorithmic_bytes(M, d, I), fw_avg
+        bound, kpeak, kpeak_src, kunit, kwork = "hbm", peak, peak_src, "GB/s", kbytes
     else:
-        kname, kbytes, kms = "gateup_stream", gateup_bytes(M, d, I), gu_avg
-    k_achieved = kbytes / (kms / 1e3) / 1e9
+        kname, kbytes, kms = "gate-up (fmlp_gate_up_swiglu)", gateup_bytes(M, d, I), gu_avg
+        # tensor-bound when the gate-up's intensity exceeds the measured ridge point
+        if gu_flops / kbytes > tpeak * 1e12 / (peak * 1e9):
+            bound, kpeak, kpeak_src, kunit, kwork = "tensor", tpeak, tpeak_src, "TFLOP/s", gu_flops
+        else:
+            bound, kpeak, kpeak_src, kunit, kwork = "hbm", peak, peak_src, "GB/s", kbytes
+    k_achieved = kwork / (kms / 1e3) / (1e12 if kunit == "TFLOP/s" else 1e9)
     traffic = recorded_traffic(kname, w.name)
 
     if rank == 0:
@@ -444,11 +456,12 @@ def run_ours(args) -> None:
             "data": "synthetic", "config": config_of(w, args),
             "hbm_frac": round(gbs / world / peak, 4),
             "tokens_per_s_per_layer": round(tok_per_s_layer, 1),
-            "roofline": {"bound": "hbm", "kernel": kname,
-                         "achieved": round(k_achieved, 2), "peak": peak, "peak_source": peak_src,
-                         "unit": "GB/s", "frac": round(k_achieved / peak, 4),
-                         "traffic": traffic, "algorithmic_bytes_per_launch": kbytes,
-                         "avg_launch_ms": round(kms, 5)},
+            "roofline": {"bound": bound, "kernel": kname,
+                         "achieved": round(k_achieved, 2), "peak": kpeak,
+                         "peak_source": kpeak_src, "unit": kunit,
+                         "frac": round(k_achieved / kpeak, 4), "traffic": traffic,
+                         "algorithmic_per_launch": kwork, "avg_launch_ms": round(kms, 5)},
+            "tflops": round(6 * M * d * I * L * args.steps * world / (elapsed_ms / 1e3) / 1e12, 2),
             "kernels": {"fmlp_forward_ms": round(fw_avg, 5),
                         "gateup_stream_ms": round(gu_avg, 5),
                         "gateup_stream_GBps": round(gateup_bytes(M, d, I) / (gu_avg / 1e3) / 1e9, 2),

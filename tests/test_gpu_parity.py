@@ -365,3 +365,53 @@ def test_maximum_and_minimum_sizes(fm, M, d, I):
     got = run_forward(fm, p, T=8, residual=True)
     assert_parity(got, oracle_out(p, residual=True), oracle_out(p, residual=True,
                                                                intermediate="bf16"))
+
+
+# ----------------------------------------------------------------------------
+# Tensor-core path (M > 4, d and I multiples of 64, T in {8, 16})
+# ----------------------------------------------------------------------------
+
+TC_CASES = [
+    (8, 512, 512, 16, False),     # 64 (tile, k-block) units: every tile split over CTAs
+    (5, 256, 1024, 8, True),
+    (16, 768, 1536, 16, True),
+    (33, 1024, 2048, 8, False),
+    (100, 512, 768, 16, True),
+    (129, 256, 512, 16, False),   # two token tiles, ragged
+    (300, 384, 640, 8, True),     # three token tiles (gate-up), two (down)
+]
+
+
+@pytest.mark.parametrize("M,d,I,T,residual", TC_CASES,
+                         ids=[f"M{c[0]}-d{c[1]}-I{c[2]}-T{c[3]}" for c in TC_CASES])
+def test_tensor_core_path(fm, M, d, I, T, residual):
+    p = wl.make_problem(M, d, I, sigma=0.03, seed=M + d + I, residual=residual)
+    got = run_forward(fm, p, T=T, residual=residual)
+    ref = oracle_out(p, residual=residual)
+    assert_parity(got, ref, oracle_out(p, residual=residual, intermediate="bf16"))
+
+
+def test_tensor_core_stage_calls(fm):
+    """The stage calls take the tensor path too: a from the gate-up GEMM, then
+    the down GEMM, against the oracle's intermediate and output."""
+    M, d, I, T = 24, 512, 1024, 16
+    p = wl.make_problem(M, d, I, sigma=0.03, seed=77)
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in p.items()}
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    a = torch.empty(M, I, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_gate_up_swiglu(g["x"], g["gamma"], EPS, packed, T, a, ws)
+    out = torch.empty(M, d, dtype=torch.float32, device=dev)
+    fm.fmlp_down_proj(a, g["W_down"], out, ws)
+    torch.cuda.synchronize()
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+    b = {k: bits(v) for k, v in p.items()}
+    h = oracle.rmsnorm(oracle.decode_bf16(b["x"]), oracle.decode_bf16(b["gamma"]), EPS)
+    a_ref = oracle.swiglu_intermediate(h, oracle.decode_bf16(b["W_gate"]),
+                                       oracle.decode_bf16(b["W_up"]))
+    a_got = oracle.decode_bf16(bits(a))
+    assert errors(a_got, a_ref)[0] <= 2.5e-3
+    assert (a_got != oracle.round_to_bf16(a_ref)).mean() < 1e-2
+    assert_parity(out.cpu().double().numpy(), oracle_out(p), oracle_out(p, intermediate="bf16"))

@@ -45,10 +45,11 @@ def test_noalloc_rejects_oversize_and_invalid_requests():
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("M,d,I,residual", [(1, 3072, 8192, False), (4, 256, 688, True),
-                                            (7, 1024, 2064, True), (128, 512, 1024, False)])
+                                            (7, 1024, 2064, True), (12, 512, 1024, False)])
 def test_noalloc_matches_workspace_entry_point(cuda_device, M, d, I, residual):
     import token_phase_swiglu_b200 as fm
     dev = cuda_device
+    assert fm.fmlp_workspace_bytes(M, d, I) <= fm.NOALLOC_SCRATCH_BYTES
     p = wl.make_problem(M, d, I, sigma=0.02, seed=31 + M, residual=residual)
     g = {k: v.to(dev) for k, v in p.items()}
     res = g["residual"] if residual else None

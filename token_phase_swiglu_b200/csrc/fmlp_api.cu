@@ -29,6 +29,20 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }  // N
 
 inline uint32_t* status_word(void* workspace) { return (uint32_t*)workspace; }
 
+// The tensor-core path takes token counts above the fused decode kernel's range.
+bool use_tc(int64_t M, int64_t d, int64_t I, int T) { return M > 4 && tc_supported(M, d, I, T); }
+
+TcWorkspace tc_workspace(void* workspace, const WorkspaceLayout& L) {
+  char* w = (char*)workspace;
+  TcWorkspace t;
+  t.b_hl = w + L.b_hl;
+  t.rinv = (float*)(w + L.rinv);
+  t.partials = (float*)(w + L.partials);
+  t.counters = (uint32_t*)(w + L.counters);
+  t.status = status_word(workspace);
+  return t;
+}
+
 fmlp_status cuda_fail(cudaError_t e) {
   g_last_cuda_error = (int)e;
   return FMLP_ERR_CUDA;
@@ -93,6 +107,17 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
   off += align256((size_t)M * (size_t)I * 2);
   L.acc = off;
   off += align256((size_t)(M < 4 ? M : 4) * (size_t)d * 4);
+  if (M > 4) {
+    const TcSizes z = tc_sizes(M, d, I, kTcMaxCtas);
+    L.b_hl = off;
+    off += align256(z.b_hl);
+    L.rinv = off;
+    off += align256(z.rinv);
+    L.partials = off;
+    off += align256(z.partials);
+    L.counters = off;
+    off += align256(z.counters);
+  }
   L.total = off;
   return L;
 }
@@ -171,8 +196,14 @@ fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* gamma, flo
   const DeviceInfo* dev = nullptr;
   st = device_for_launch(&dev);
   if (st != FMLP_OK) return st;
-  cudaError_t e = launch_gateup_stream(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a,
-                                       status_word(workspace), *dev, (cudaStream_t)stream);
+  cudaError_t e;
+  if (use_tc(M, d, I, tile_T))
+    e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a,
+                         tc_workspace(workspace, workspace_layout(M, d, I)), *dev,
+                         (cudaStream_t)stream);
+  else
+    e = launch_gateup_stream(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a,
+                             status_word(workspace), *dev, (cudaStream_t)stream);
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
 }
 
@@ -189,8 +220,14 @@ fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t
   const DeviceInfo* dev = nullptr;
   st = device_for_launch(&dev);
   if (st != FMLP_OK) return st;
-  cudaError_t e = launch_down_stream(a, M, W_down, d, I, residual, out, status_word(workspace),
-                                     *dev, (cudaStream_t)stream);
+  cudaError_t e;
+  if (use_tc(M, d, I, 16))
+    e = launch_tc_down(a, M, W_down, d, I, residual, out,
+                       tc_workspace(workspace, workspace_layout(M, d, I)), *dev,
+                       (cudaStream_t)stream);
+  else
+    e = launch_down_stream(a, M, W_down, d, I, residual, out, status_word(workspace), *dev,
+                           (cudaStream_t)stream);
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
 }
 
@@ -220,6 +257,10 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
     uint32_t* done = (uint32_t*)((char*)workspace + L.done);
     e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out, acc,
                             done, status, *dev, s);
+  } else if (use_tc(M, d, I, tile_T)) {
+    const TcWorkspace tw = tc_workspace(workspace, L);
+    e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, tw, *dev, s);
+    if (e == cudaSuccess) e = launch_tc_down(a, M, W_down, d, I, residual, out, tw, *dev, s);
   } else {
     e = launch_gateup_stream(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, status, *dev, s);
     if (e == cudaSuccess)

@@ -29,6 +29,7 @@ struct WorkspaceLayout {
   size_t done = 128;     // uint32 finished-CTA counter (fused kernel)
   size_t a = 0;          // bf16 [M x I] intermediate
   size_t acc = 0;        // f32 [min(M,4) x d] accumulator (fused kernel)
+  size_t b_hl = 0, rinv = 0, partials = 0, counters = 0;  // tensor-core path (M > 4)
   size_t total = 0;
 };
 WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I);
@@ -65,6 +66,27 @@ cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, flo
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
                                 const void* residual, float* out, float* acc, uint32_t* done,
                                 uint32_t* status, const DeviceInfo& dev, cudaStream_t stream);
+
+// Tensor-core path (tcgen05, csrc/tc.cu) for M above the decode range.
+constexpr int kTcMaxCtas = 160;  // workspace sizing bound on the grid (>= SMs of a B200)
+struct TcWorkspace {
+  void* b_hl;          // bf16 token-tiled [hi; lo] rows of x*gamma
+  float* rinv;         // [M] 1/RMS
+  float* partials;     // stream-K partial accumulators
+  uint32_t* counters;  // per-tile arrival counters (zero between calls)
+  uint32_t* status;
+};
+struct TcSizes {
+  size_t b_hl = 0, rinv = 0, partials = 0, counters = 0;
+};
+TcSizes tc_sizes(int64_t M, int64_t d, int64_t I, int sm_count);
+bool tc_supported(int64_t M, int64_t d, int64_t I, int T);
+cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float eps,
+                             const void* P, int T, int64_t d, int64_t I, void* a,
+                             const TcWorkspace& ws, const DeviceInfo& dev, cudaStream_t stream);
+cudaError_t launch_tc_down(const void* a, int64_t M, const void* W_down, int64_t d, int64_t I,
+                           const void* residual, float* out, const TcWorkspace& ws,
+                           const DeviceInfo& dev, cudaStream_t stream);
 
 // out[m, n] = sum_i W_down[n, i] a[m, i] (+ residual), same streaming scheme.
 cudaError_t launch_down_stream(const void* a, int64_t M, const void* W_down, int64_t d,

@@ -1,0 +1,717 @@
+// Tensor-core path (tcgen05 / TMEM) for token counts above the decode range.
+//
+// The gate-up contraction and the down projection of the MLP block
+// ("FastTPS: An Optimized Method for LLM Token Phase for AI Accelerators",
+// xllm-io review, section 三 Eq(1), Figure 4) as swap-AB GEMMs:
+//
+//     D[r, n] = sum_k A[r, k] B[n, k]
+//
+// with the weights as A (128 rows per MMA tile, M of the MMA) and the token
+// rows as B (N of the MMA, 16..256).  For the gate-up step B holds, per token
+// tile of Mt tokens, the rows hi(x*gamma) then lo(x*gamma): x*gamma has at
+// most 16 significant bits, so hi + lo (two bf16) is exact and the MMA sees
+// the activations at f32 precision; the epilogue adds the two halves of D.
+// r = 1/RMS is applied in the epilogue, as in the CUDA-core path.
+//
+// Per CTA (one per SM, 192 threads):
+//   warp 0     TMA producer: one 16 KB A box + one B box per 64-wide k-block
+//              into a ring of shared-memory stages (128-byte swizzle);
+//   warp 1     TMEM owner and MMA issuer (tcgen05.mma kind::f16, f32
+//              accumulators double-buffered in TMEM, tcgen05.commit frees
+//              stages and publishes accumulators);
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//              lanes 32*(w%4)..+31), SwiGLU or residual add, stores.
+// Work is split "stream-K": the (tile, k-block) units are cut evenly over the
+// CTAs, so a tile may be shared by two or more CTAs; each writes its partial
+// accumulator to the workspace and the last one to arrive (tile counter) sums
+// them and runs the epilogue.  Nobody waits on another CTA.
+// Every mbarrier wait is bounded; on expiry the CTA flags the status word,
+// waits for its own copies and MMAs, frees its TMEM and returns.
+#include "common.cuh"
+#include "internal.h"
+#include "tmap.h"
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <set>
+
+namespace fmlp {
+namespace {
+
+constexpr int kTcThreads = 192;
+constexpr int kBM = 128;        // A rows per tile (MMA M)
+constexpr int kBK = 64;         // k-block: one 128-byte swizzle atom of bf16
+constexpr int kATileBytes = kBM * kBK * 2;
+constexpr int kMaxStages = 12;
+constexpr uint64_t kDrainNs = 1000000000ull;
+
+enum Epi { kEpiSwiGLU = 0, kEpiDown = 1 };
+
+// ---------------------------------------------------------------------------
+// tcgen05 wrappers
+// ---------------------------------------------------------------------------
+// Shared-memory matrix descriptor: K-major tile of rows x 128 bytes with the
+// 128-byte swizzle (8-row atoms of 1024 bytes, stride 1024 bytes between atoms).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address (16-byte units)
+  d |= (uint64_t)1 << 16;                    // leading offset: unused for swizzled K-major
+  d |= (uint64_t)(1024 >> 4) << 32;          // stride offset between 8-row atoms
+  d |= (uint64_t)1 << 46;                    // descriptor version
+  d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> f32, A and B K-major, M = 128, N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(kBM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                   "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// 32 lanes x 8 consecutive 32-bit columns; thread i of the warp gets lane
+// (32 * (warp % 4) + i), columns col..col+7.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Barrier of the four epilogue warps that also ORs a failure flag, so that a
+// timeout in any of them makes all of them leave together.
+__device__ __forceinline__ bool epilogue_barrier_any(bool failed) {
+  uint32_t any;
+  asm volatile(
+      "{\n .reg .pred q, r;\n setp.ne.u32 q, %1, 0;\n"
+      " bar.red.or.pred r, 2, 128, q;\n selp.u32 %0, 1, 0, r;\n}"
+      : "=r"(any)
+      : "r"((uint32_t)failed)
+      : "memory");
+  return any != 0;
+}
+
+// ---------------------------------------------------------------------------
+// Stream-K schedule
+// ---------------------------------------------------------------------------
+struct Sched {
+  int KB;      // k-blocks per tile
+  int tiles;   // row tiles x token tiles
+  int ntok;    // token tiles (tile index = row_tile * ntok + token_tile)
+  int ctas;    // grid size
+  __device__ __forceinline__ int64_t units() const { return (int64_t)tiles * KB; }
+  // unit range of CTA c
+  __device__ __forceinline__ void range(int c, int64_t& u0, int64_t& u1) const {
+    const int64_t U = units(), per = U / ctas, rem = U % ctas;
+    u0 = c * per + (c < rem ? (int64_t)c : rem);
+    u1 = u0 + per + (c < rem ? 1 : 0);
+  }
+  __device__ __forceinline__ int cta_of(int64_t u) const {
+    const int64_t U = units(), per = U / ctas, rem = U % ctas;
+    const int64_t big = rem * (per + 1);
+    return u < big ? (int)(u / (per + 1)) : (int)(rem + (u - big) / per);
+  }
+};
+
+// Segment s of this CTA's range: tile t, k-blocks [kb0, kb1).  Returns false past the end.
+__device__ __forceinline__ bool segment(const Sched& S, int64_t u0, int64_t u1, int s, int& t,
+                                        int& kb0, int& kb1) {
+  if (u0 >= u1) return false;
+  const int t0 = (int)(u0 / S.KB);
+  t = t0 + s;
+  const int64_t tb = (int64_t)t * S.KB;
+  if (tb >= u1) return false;
+  kb0 = (int)(max(u0, tb) - tb);
+  kb1 = (int)(min(u1, tb + S.KB) - tb);
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel
+// ---------------------------------------------------------------------------
+struct TcParams {
+  CUtensorMap a_map;   // A [rows x K] bf16, box 64 x 128, 128-byte swizzle
+  CUtensorMap b_map;   // B [token-tile rows x K] bf16, box 64 x N, 128-byte swizzle
+  Sched sched;
+  int epi;             // kEpiSwiGLU or kEpiDown
+  int N;               // MMA N (columns of D)
+  int Mt;              // tokens per token tile
+  int M;               // tokens
+  int rows;            // valid A rows (2I packed rows, or d)
+  int T;               // interleave tile (SwiGLU)
+  int I, d;
+  int stages, stage_bytes, b_bytes;
+  uint32_t tmem_cols;  // allocated TMEM columns (2 x N rounded up to a power of two)
+  const float* rinv;   // [M] 1/RMS per token (SwiGLU)
+  __nv_bfloat16* a_out;             // SwiGLU output a [M x I]
+  float* out;                       // down output [M x d]
+  const __nv_bfloat16* residual;    // [M x d] or null
+  float* partials;     // [ctas][2][N][128] f32
+  uint32_t* counters;  // [tiles] arrivals (zero between calls)
+  uint32_t* status;
+  uint64_t wait_ns;
+  int drop_last;
+};
+
+struct TcShared {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t mma_done;   // abort path: all issued MMAs have completed
+  uint32_t tmem_base;
+  int abort;
+  int last;
+  int k_issued;        // stages issued by the producer
+};
+
+__device__ __forceinline__ void tc_flag(TcShared* sh, uint32_t* status) {
+  sh->abort = 1;
+  atomicOr(status, kStatusTimeout);
+}
+
+// Epilogue of CW logical columns [col0, col0 + CW) of one finished tile
+// (warps 2-5; vals[j] = D[row, col0 + j], hi + lo already summed).
+template <int CW>
+__device__ __forceinline__ void epilogue_columns(const TcParams& p, int tile, const float (&vals)[CW],
+                                                 int col0, int r_local) {
+  const int rt = tile / p.sched.ntok, tt = tile % p.sched.ntok;
+  const int row = rt * kBM + r_local;
+  if (p.epi == kEpiDown) {
+    const int n = row;
+#pragma unroll
+    for (int j = 0; j < CW; ++j) {
+      const int m = tt * p.Mt + col0 + j;
+      if (m < p.M && n < p.d) {
+        float o = vals[j];
+        if (p.residual) o += __bfloat162float(p.residual[(int64_t)m * p.d + n]);
+        p.out[(int64_t)m * p.d + n] = o;
+      }
+    }
+    return;
+  }
+  // SwiGLU: within a 2T-row interleave tile rows [0,T) are gate, [T,2T) up;
+  // the partner row is lane ^ T (T in {8, 16}).  The gate lane finishes the
+  // first half of the chunk's tokens, the up lane the second half.
+  constexpr int H = CW / 2;
+  const int T = p.T;
+  const bool is_gate = (row % (2 * T)) < T;
+  float g[H], u[H];
+#pragma unroll
+  for (int j = 0; j < H; ++j) {
+    const float send = is_gate ? vals[H + j] : vals[j];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, T);
+    g[j] = is_gate ? vals[j] : recv;
+    u[j] = is_gate ? recv : vals[H + j];
+  }
+  const int pair = (row / (2 * T)) * T + (row % T);
+  const int tok0 = tt * p.Mt + col0 + (is_gate ? 0 : H);
+  if (row < p.rows && pair < p.I) {
+#pragma unroll
+    for (int j = 0; j < H; ++j) {
+      const int m = tok0 + j;
+      if (m < p.M) {
+        const float r = p.rinv[m];
+        p.a_out[(int64_t)m * p.I + pair] = __float2bfloat16_rn(silu_mul(g[j] * r, u[j] * r));
+      }
+    }
+  }
+}
+
+// Finish one tile: sum the accumulator (hi + lo for SwiGLU) with the other
+// contributors' partials, CW logical columns at a time.
+template <int CW>
+__device__ void finish_tile(const TcParams& p, int t, uint32_t tb, bool whole, int c_first,
+                            int c_last, int r_local) {
+  const int ncol = p.epi == kEpiSwiGLU ? p.Mt : p.N;
+  for (int c0 = 0; c0 < ncol; c0 += CW) {
+    float vals[CW];
+#pragma unroll
+    for (int c = 0; c < CW; c += 8) {
+      float v[8];
+      tmem_ld8(tb + c0 + c, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) vals[c + j] = v[j];
+      if (p.epi == kEpiSwiGLU) {
+        tmem_ld8(tb + p.Mt + c0 + c, v);  // lo half of x*gamma
+#pragma unroll
+        for (int j = 0; j < 8; ++j) vals[c + j] += v[j];
+      }
+    }
+    if (!whole) {
+      for (int cc = c_first; cc <= c_last; ++cc) {
+        if (cc == (int)blockIdx.x) continue;
+        int64_t cu0, cu1;
+        p.sched.range(cc, cu0, cu1);
+        const int slot = (t == (int)(cu0 / p.sched.KB)) ? 0 : 1;
+        const float* part = p.partials + ((size_t)cc * 2 + slot) * (size_t)p.N * kBM;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          vals[j] += __ldcg(part + (size_t)(c0 + j) * kBM + r_local);
+          if (p.epi == kEpiSwiGLU) vals[j] += __ldcg(part + (size_t)(p.Mt + c0 + j) * kBM + r_local);
+        }
+      }
+    }
+    epilogue_columns<CW>(p, t, vals, c0, r_local);
+  }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__ TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ TcShared sh;
+  // stages start at a 1024-byte boundary (128-byte swizzle atoms)
+  uint8_t* stage0 = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int64_t u0, u1;
+  p.sched.range(blockIdx.x, u0, u1);
+  int nseg = 0, nk = 0;
+  {
+    int t, a, b;
+    while (segment(p.sched, u0, u1, nseg, t, a, b)) {
+      nk += b - a;
+      ++nseg;
+    }
+  }
+
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < p.stages; ++j) {
+      mbar_init(&sh.full[j], 1);
+      mbar_init(&sh.empty[j], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&sh.acc_full[j], 1);
+      mbar_init(&sh.acc_empty[j], 4);
+    }
+    mbar_init(&sh.mma_done, 1);
+    sh.abort = 0;
+    sh.k_issued = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sh.tmem_base, p.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  grid_launch_dependents();
+  const uint32_t tmem = sh.tmem_base;
+  volatile int* abort = &sh.abort;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    // The weights (A) do not depend on the previous kernel: the first ring's
+    // worth of A tiles is requested before the dependency wait; the
+    // activations (B) only after it.
+    if (lane == 0) {
+      const uint64_t pol_a = evict_first_policy();
+      uint64_t pol_b;
+      asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_b));
+      const int brow_mul = p.epi == kEpiSwiGLU ? 2 * p.Mt : p.Mt;
+      int early_kb[kMaxStages], early_tt[kMaxStages];
+      const int n_early = min(nk, p.stages) - (p.drop_last && nk <= p.stages ? 1 : 0);
+      int k = 0;
+      bool ok = true;
+      for (int s = 0; s < nseg && ok && !*abort; ++s) {
+        int t, kb0, kb1;
+        segment(p.sched, u0, u1, s, t, kb0, kb1);
+        const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
+        for (int kb = kb0; kb < kb1; ++kb, ++k) {
+          if (p.drop_last && k == nk - 1) {
+            ok = false;
+            break;
+          }
+          const int slot = k % p.stages;
+          uint8_t* a_dst = stage0 + (size_t)slot * p.stage_bytes;
+          uint8_t* b_dst = a_dst + kATileBytes;
+          if (k >= p.stages) {
+            if (k == p.stages) {
+              // activations of the early stages, now that they are written
+              grid_dependency_wait();
+              for (int e = 0; e < n_early; ++e)
+                tma_load_2d(stage0 + (size_t)e * p.stage_bytes + kATileBytes, &p.b_map,
+                            early_kb[e] * kBK, early_tt[e] * brow_mul, &sh.full[e], pol_b);
+            }
+            if (!mbar_wait_bounded(&sh.empty[slot], (uint32_t)(((k / p.stages) - 1) & 1),
+                                   p.wait_ns, abort)) {
+              tc_flag(&sh, p.status);
+              ok = false;
+              break;
+            }
+          }
+          mbar_arrive_expect_tx(&sh.full[slot], (uint32_t)(kATileBytes + p.b_bytes));
+          tma_load_2d(a_dst, &p.a_map, kb * kBK, rt * kBM, &sh.full[slot], pol_a);
+          if (k < p.stages) {
+            early_kb[k] = kb;
+            early_tt[k] = tt;
+          } else {
+            tma_load_2d(b_dst, &p.b_map, kb * kBK, tt * brow_mul, &sh.full[slot], pol_b);
+          }
+          sh.k_issued = k + 1;
+        }
+      }
+      if (k <= p.stages && k > 0) {
+        // the whole range fit in the first ring: its activations are still owed
+        grid_dependency_wait();
+        for (int e = 0; e < k; ++e)
+          tma_load_2d(stage0 + (size_t)e * p.stage_bytes + kATileBytes, &p.b_map,
+                      early_kb[e] * kBK, early_tt[e] * brow_mul, &sh.full[e], pol_b);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    grid_dependency_wait();  // B is written by the previous kernel
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(p.N);
+      int k = 0;
+      bool ok = true;
+      for (int s = 0; s < nseg && ok; ++s) {
+        int t, kb0, kb1;
+        segment(p.sched, u0, u1, s, t, kb0, kb1);
+        const int buf = s & 1;
+        if (!mbar_wait_bounded(&sh.acc_empty[buf], (uint32_t)(((s >> 1) & 1) ^ 1), p.wait_ns,
+                               abort)) {
+          tc_flag(&sh, p.status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * p.N);
+        for (int kb = kb0; kb < kb1; ++kb, ++k) {
+          const int slot = k % p.stages;
+          if (!mbar_wait_bounded(&sh.full[slot], (uint32_t)((k / p.stages) & 1), p.wait_ns,
+                                 abort)) {
+            tc_flag(&sh, p.status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stage0 + (size_t)slot * p.stage_bytes);
+          const uint32_t b_addr = a_addr + kATileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16(d_tmem, sw128_desc(a_addr + kk * 32), sw128_desc(b_addr + kk * 32), idesc,
+                     (kb > kb0 || kk > 0) ? 1u : 0u);
+          mma_commit(&sh.empty[slot]);  // stage reusable once these MMAs finish
+        }
+        if (ok) mma_commit(&sh.acc_full[buf]);
+      }
+      // every MMA issued so far has completed once this commit arrives
+      mma_commit(&sh.mma_done);
+      mbar_wait_bounded(&sh.mma_done, 0, kDrainNs, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2-5) ----------------
+    const int q = warp & 3;                  // TMEM lane quadrant of this warp
+    const int r_local = 32 * q + lane;       // accumulator row = TMEM lane
+    const int et = threadIdx.x - 64;         // 0..127
+    const int ncol = p.epi == kEpiSwiGLU ? p.Mt : p.N;  // logical columns (hi + lo summed)
+    grid_dependency_wait();  // 1/RMS and the residual come from earlier kernels
+    for (int s = 0; s < nseg; ++s) {
+      int t, kb0, kb1;
+      segment(p.sched, u0, u1, s, t, kb0, kb1);
+      const int buf = s & 1;
+      const bool got =
+          mbar_wait_bounded(&sh.acc_full[buf], (uint32_t)((s >> 1) & 1), p.wait_ns, abort);
+      if (!got && lane == 0) tc_flag(&sh, p.status);
+      if (epilogue_barrier_any(!got)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.N);
+      const bool whole = kb0 == 0 && kb1 == p.sched.KB;
+      const int c_first = p.sched.cta_of((int64_t)t * p.sched.KB);
+      const int c_last = p.sched.cta_of((int64_t)t * p.sched.KB + p.sched.KB - 1);
+      bool finalize = whole;
+      if (!whole) {
+        // this CTA's partial: slot 0 if the tile is where its range starts, else 1
+        const int slot = (t == (int)(u0 / p.sched.KB)) ? 0 : 1;
+        float* part = p.partials + ((size_t)blockIdx.x * 2 + slot) * (size_t)p.N * kBM;
+        for (int c = 0; c < p.N; c += 8) {
+          float v[8];
+          tmem_ld8(tb + c, v);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) __stcg(part + (size_t)(c + j) * kBM + r_local, v[j]);
+        }
+        __threadfence();
+        named_barrier_sync(1, 128);
+        if (et == 0) sh.last = atomicAdd(p.counters + t, 1u) == (uint32_t)(c_last - c_first);
+        named_barrier_sync(1, 128);
+        finalize = sh.last;
+        if (finalize) __threadfence();
+      }
+      if (finalize) {
+        if (ncol >= 32) finish_tile<32>(p, t, tb, whole, c_first, c_last, r_local);
+        else if (ncol >= 16) finish_tile<16>(p, t, tb, whole, c_first, c_last, r_local);
+        else finish_tile<8>(p, t, tb, whole, c_first, c_last, r_local);
+        if (!whole && et == 0) atomicExch(p.counters + t, 0u);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && sh.abort) {
+    for (int k = max(0, sh.k_issued - p.stages); k < sh.k_issued; ++k)
+      mbar_wait_bounded(&sh.full[k % p.stages], (uint32_t)((k / p.stages) & 1), kDrainNs, nullptr);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Prologue: B operand of the gate-up GEMM and 1/RMS per token.
+// One CTA per token slot of the padded token tiles: rows [2Mt*j + i] = hi and
+// [2Mt*j + Mt + i] = lo of token m = Mt*j + i (zeros for padding slots).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict__ x,
+                                                 const __nv_bfloat16* __restrict__ gamma,
+                                                 float eps, int M, int d, int Mt,
+                                                 __nv_bfloat16* __restrict__ b_hl,
+                                                 float* __restrict__ rinv) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int slot = blockIdx.x;
+  const int j = slot / Mt, i = slot % Mt;
+  const int m = slot;
+  __nv_bfloat16* hi = b_hl + ((int64_t)2 * Mt * j + i) * d;
+  __nv_bfloat16* lo = hi + (int64_t)Mt * d;
+  __shared__ float red[8];
+  float ss = 0.f;
+  for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
+    uint4 xv = make_uint4(0, 0, 0, 0);
+    if (m < M) xv = ld_keep(x + (int64_t)m * d + (int64_t)v * 8);
+    const uint4 gv = ld_keep(gamma + (int64_t)v * 8);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = bf16lo(xw[e]), x1 = bf16hi(xw[e]);
+      ss = fmaf(x0, x0, ss);
+      ss = fmaf(x1, x1, ss);
+      const float s0 = x0 * bf16lo(gw[e]), s1 = x1 * bf16hi(gw[e]);  // exact in f32
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(s0), h1 = __float2bfloat16_rn(s1);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(s0 - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(s1 - __bfloat162float(h1));
+      hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    reinterpret_cast<uint4*>(hi)[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    reinterpret_cast<uint4*>(lo)[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0 && m < M) {
+    float t = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    rinv[m] = 1.0f / sqrtf(t / (float)d + eps);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+struct TcPlan {
+  int N = 0, Mt = 0, ntok = 0, stages = 0, stage_bytes = 0, b_bytes = 0;
+  uint32_t tmem_cols = 0;
+  size_t smem = 0;
+};
+
+uint32_t pow2_at_least(uint32_t n) {
+  uint32_t c = 32;
+  while (c < n) c <<= 1;
+  return c;
+}
+
+TcPlan make_tc_plan(int epi, int64_t M, const DeviceInfo& dev) {
+  TcPlan pl;
+  if (epi == kEpiSwiGLU) {
+    pl.Mt = (int)std::min<int64_t>(128, (M + 7) / 8 * 8);
+    pl.N = 2 * pl.Mt;
+  } else {
+    pl.Mt = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
+    pl.N = pl.Mt;
+  }
+  pl.ntok = (int)((M + pl.Mt - 1) / pl.Mt);
+  pl.b_bytes = pl.N * kBK * 2;
+  pl.stage_bytes = (kATileBytes + pl.b_bytes + 1023) / 1024 * 1024;
+  const size_t budget = (size_t)dev.max_smem_optin - 2048 - 1024;  // static + alignment slack
+  pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
+  pl.smem = (size_t)pl.stages * pl.stage_bytes + 1024;
+  pl.tmem_cols = pow2_at_least((uint32_t)(2 * pl.N));
+  return pl;
+}
+
+cudaError_t allow_tc_smem(const DeviceInfo& dev) {
+  static std::mutex mu;
+  static std::set<int> done;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count(dev.device)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dev.max_smem_optin - 2048);
+  if (e == cudaSuccess) done.insert(dev.device);
+  return e;
+}
+
+cudaError_t launch_tc(const TcParams& p, const TcPlan& pl, const DeviceInfo& dev,
+                      cudaStream_t stream) {
+  cudaError_t e = allow_tc_smem(dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.sched.ctas);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, tc_gemm, p);
+  if (e == cudaSuccess) note_launches(1);
+  return e;
+}
+
+void fill_common(TcParams& p, const TcPlan& pl, int epi, int64_t M, int rows, int K,
+                 const TcWorkspace& ws, const DeviceInfo& dev) {
+  (void)epi;
+  p.epi = epi;
+  p.N = pl.N;
+  p.Mt = pl.Mt;
+  p.M = (int)M;
+  p.rows = rows;
+  p.stages = pl.stages;
+  p.stage_bytes = pl.stage_bytes;
+  p.b_bytes = pl.b_bytes;
+  p.tmem_cols = pl.tmem_cols;
+  p.sched.KB = (K + kBK - 1) / kBK;
+  p.sched.ntok = pl.ntok;
+  p.sched.tiles = ((rows + kBM - 1) / kBM) * pl.ntok;
+  p.sched.ctas = (int)std::min<int64_t>(
+      {(int64_t)p.sched.tiles * p.sched.KB, (int64_t)dev.sm_count, (int64_t)kTcMaxCtas});
+  p.partials = ws.partials;
+  p.counters = ws.counters;
+  p.status = ws.status;
+  p.wait_ns = wait_timeout_ns();
+  p.drop_last = fault_injection();
+}
+
+}  // namespace
+
+TcSizes tc_sizes(int64_t M, int64_t d, int64_t I, int sm_count) {
+  if (M < 1) return TcSizes();
+  TcSizes z;
+  const int Mt_g = (int)std::min<int64_t>(128, (M + 7) / 8 * 8);
+  const int ntok_g = (int)((M + Mt_g - 1) / Mt_g);
+  z.b_hl = (size_t)ntok_g * 2 * Mt_g * d * 2;
+  z.rinv = (size_t)M * 4;
+  const int N_max = std::max(2 * Mt_g, (int)std::min<int64_t>(256, (M + 15) / 16 * 16));
+  z.partials = (size_t)sm_count * 2 * N_max * kBM * 4;
+  const int64_t tiles_g = ((2 * I + kBM - 1) / kBM) * ntok_g;
+  const int Mt_d = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
+  const int64_t tiles_d = ((d + kBM - 1) / kBM) * ((M + Mt_d - 1) / Mt_d);
+  z.counters = (size_t)std::max(tiles_g, tiles_d) * 4;
+  return z;
+}
+
+bool tc_supported(int64_t M, int64_t d, int64_t I, int T) {
+  return M >= 1 && d % 64 == 0 && I % 64 == 0 && (T == 8 || T == 16);
+}
+
+cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float eps,
+                             const void* P, int T, int64_t d, int64_t I, void* a,
+                             const TcWorkspace& ws, const DeviceInfo& dev, cudaStream_t stream) {
+  const TcPlan pl = make_tc_plan(kEpiSwiGLU, M, dev);
+  // prologue: hi/lo split of x * gamma into the token-tiled B operand, and 1/RMS
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(pl.ntok * pl.Mt));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, act_split, (const __nv_bfloat16*)x,
+                                       (const __nv_bfloat16*)gamma, eps, (int)M, (int)d, pl.Mt,
+                                       (__nv_bfloat16*)ws.b_hl, ws.rinv);
+    if (e != cudaSuccess) return e;
+    note_launches(1);
+  }
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  const int rows = (int)(2 * I);
+  cudaError_t e = encode_tmap_2d_bf16(&p.a_map, P, (uint64_t)rows, (uint64_t)d, (uint64_t)d * 2,
+                                      kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e == cudaSuccess)
+    e = encode_tmap_2d_bf16(&p.b_map, ws.b_hl, (uint64_t)pl.ntok * 2 * pl.Mt, (uint64_t)d,
+                            (uint64_t)d * 2, (uint32_t)pl.N, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  fill_common(p, pl, kEpiSwiGLU, M, rows, (int)d, ws, dev);
+  p.T = T;
+  p.I = (int)I;
+  p.d = (int)d;
+  p.rinv = ws.rinv;
+  p.a_out = (__nv_bfloat16*)a;
+  return launch_tc(p, pl, dev, stream);
+}
+
+cudaError_t launch_tc_down(const void* a, int64_t M, const void* W_down, int64_t d, int64_t I,
+                           const void* residual, float* out, const TcWorkspace& ws,
+                           const DeviceInfo& dev, cudaStream_t stream) {
+  const TcPlan pl = make_tc_plan(kEpiDown, M, dev);
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  cudaError_t e = encode_tmap_2d_bf16(&p.a_map, W_down, (uint64_t)d, (uint64_t)I,
+                                      (uint64_t)I * 2, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e == cudaSuccess)
+    e = encode_tmap_2d_bf16(&p.b_map, a, (uint64_t)M, (uint64_t)I, (uint64_t)I * 2,
+                            (uint32_t)pl.N, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  fill_common(p, pl, kEpiDown, M, (int)d, (int)I, ws, dev);
+  p.I = (int)I;
+  p.d = (int)d;
+  p.out = out;
+  p.residual = (const __nv_bfloat16*)residual;
+  return launch_tc(p, pl, dev, stream);
+}
+
+}  // namespace fmlp
