@@ -157,6 +157,22 @@ def dist_env():
     return rank, world, local
 
 
+def reduce_max(v: float, device=None) -> float:
+    """The maximum of `v` over all ranks (the value itself without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_step_per_rank: int, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: the bytes every replica streamed over the slowest
+    rank's device time (replicas do equal work, so weak scaling)."""
+    return bytes_per_step_per_rank * steps * world / (elapsed_ms / 1e3) / 1e9
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -302,12 +318,7 @@ def run_ours(args) -> None:
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dev)
 
     # warm-up (also the one-time library set-up, before any graph capture)
     for _ in range(max(1, args.warmup)):
@@ -355,8 +366,7 @@ def run_ours(args) -> None:
     fm_status = fm.fmlp_device_status(ws)
 
     bytes_step = L * algorithmic_bytes(M, d, I)
-    total_bytes = bytes_step * args.steps * world
-    gbs = total_bytes / (elapsed_ms / 1e3) / 1e9
+    gbs = job_gbs(bytes_step, args.steps, world, elapsed_ms)
     ms_step = elapsed_ms / args.steps
     tok_per_s_layer = M * L * args.steps * world / (elapsed_ms / 1e3)
 
@@ -417,7 +427,7 @@ def run_ours(args) -> None:
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1))
-    e2e_gbs = bytes_step * e2e_steps * world / (e2e_ms / 1e3) / 1e9
+    e2e_gbs = job_gbs(bytes_step, e2e_steps, world, e2e_ms)
 
     peaks = measured_peaks()
     if "hbm_gbs" in peaks:

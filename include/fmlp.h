@@ -79,11 +79,13 @@ FMLP_API fmlp_status fmlp_pack(const void* W_gate, const void* W_up, int64_t d, 
 
 /*
  * fmlp_workspace_bytes -- bytes of device workspace fmlp_forward needs for
- * (M, d, I).  The workspace holds a device status word, the bf16
- * intermediate a [M x I] and the control words of the fused kernel's
- * grid-wide barrier.  A workspace must be zero-filled once before its first
- * use; the library keeps its control words consistent from call to call.
- * Returns 0 for invalid sizes.
+ * (M, d, I).  The workspace holds a device status word, the fused decode
+ * kernel's completion counter and f32 accumulator, the bf16 intermediate
+ * a [M x I], and the tensor-core path's operand copy and stream-K partials.
+ * A workspace must be zero-filled before its first use and again before it
+ * serves a call with a larger d than all calls before; in between, every
+ * call (a timed-out one too) leaves it ready for the next call of any M and
+ * I.  Returns 0 for invalid sizes.
  */
 FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
 
@@ -99,8 +101,8 @@ FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
  *   W_down     : bf16 [d x I]
  *   residual   : bf16 [M x d] added to the output, or NULL
  *   out        : f32 [M x d]
- *   workspace  : >= fmlp_workspace_bytes(M, d, I) bytes, zero-filled before
- *                first use, not shared by calls that may overlap on the GPU
+ *   workspace  : >= fmlp_workspace_bytes(M, d, I) bytes, zeroed as described
+ *                there, not shared by calls that may overlap on the GPU
  *
  * Precision: x*gamma is formed exactly in f32 and the contraction keeps it at
  * f32 precision (CUDA-core path) or as an exact hi+lo bf16 pair (tensor-core

@@ -274,6 +274,29 @@ def test_side_stream_and_workspace_reuse(fm):
     assert fm.fmlp_device_status(ws) == fm.FMLP_OK
 
 
+def test_workspace_reuse_across_paths(fm):
+    """One workspace, zeroed once, serves calls of any M and I at a fixed d:
+    the fused decode kernel, the tensor-core GEMMs and the streaming kernels
+    in turn, each leaving it ready for the next."""
+    dev = torch.device("cuda:0")
+    d, T = 512, 16
+    shapes = [(12, 1024), (3, 1024), (40, 640), (1, 640), (7, 1024), (2, 1024), (9, 688),
+              (4, 640)]
+    ws = torch.zeros(max(fm.fmlp_workspace_bytes(M, d, I) for M, I in shapes),
+                     dtype=torch.uint8, device=dev)
+    for k, (M, I) in enumerate(shapes):
+        p = wl.make_problem(M, d, I, seed=70 + k, residual=k % 2 == 1)
+        g = {n: v.to(dev) for n, v in p.items()}
+        packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+        fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+        out = torch.full((M, d), float("nan"), dtype=torch.float32, device=dev)
+        fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, T, g["W_down"], out, ws,
+                        residual=g["residual"] if k % 2 == 1 else None)
+        torch.cuda.synchronize()
+        assert_parity(out.cpu().double().numpy(), oracle_out(p, residual=k % 2 == 1))
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+
+
 def test_invalid_arguments_raise(fm):
     dev = torch.device("cuda:0")
     d, I = 256, 688
@@ -379,6 +402,9 @@ TC_CASES = [
     (100, 512, 768, 16, True),
     (129, 256, 512, 16, False),   # two token tiles, ragged
     (300, 384, 640, 8, True),     # three token tiles (gate-up), two (down)
+    (24, 512, 1024, 16, True),    # 4 row sub-tiles, 16-column epilogue chunks
+    (72, 256, 512, 8, False),     # one row sub-tile, 8-column chunks, 16-column partial tail
+    (40, 640, 1280, 16, True),    # 2 row sub-tiles (gate-up), 8-column chunks
 ]
 
 

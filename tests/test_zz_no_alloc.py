@@ -8,7 +8,8 @@ buffer that the library keeps on each GPU, so the call needs no workspace.
 
 The GPU test checks it through the C ABI against fmlp_forward with a
 caller-allocated workspace, on two calls in a row (the second call finds the
-buffer as the first one left it).  This file is collected last on purpose.
+buffer as the first one left it), over shapes whose order sends a fused
+decode call with a wider d after calls that wrote the intermediate.  This file is collected last on purpose.
 """
 
 import numpy as np
@@ -45,7 +46,8 @@ def test_noalloc_rejects_oversize_and_invalid_requests():
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("M,d,I,residual", [(1, 3072, 8192, False), (4, 256, 688, True),
-                                            (7, 1024, 2064, True), (12, 512, 1024, False)])
+                                            (7, 1024, 2064, True), (12, 512, 1024, False),
+                                            (2, 2048, 1024, True)])
 def test_noalloc_matches_workspace_entry_point(cuda_device, M, d, I, residual):
     import token_phase_swiglu_b200 as fm
     dev = cuda_device

@@ -30,7 +30,9 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }  // N
 inline uint32_t* status_word(void* workspace) { return (uint32_t*)workspace; }
 
 // The tensor-core path takes token counts above the fused decode kernel's range.
-bool use_tc(int64_t M, int64_t d, int64_t I, int T) { return M > 4 && tc_supported(M, d, I, T); }
+bool use_tc(int64_t M, int64_t d, int64_t I, int T) {
+  return M > kFusedMaxM && tc_supported(M, d, I, T);
+}
 
 TcWorkspace tc_workspace(void* workspace, const WorkspaceLayout& L) {
   char* w = (char*)workspace;
@@ -39,6 +41,7 @@ TcWorkspace tc_workspace(void* workspace, const WorkspaceLayout& L) {
   t.rinv = (float*)(w + L.rinv);
   t.partials = (float*)(w + L.partials);
   t.counters = (uint32_t*)(w + L.counters);
+  t.ncounters = (int)L.ncounters;
   t.status = status_word(workspace);
   return t;
 }
@@ -103,11 +106,12 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
   L.status = off;
   L.done = off + 128;
   off += 256;
+  L.acc = off;
+  off += align256((size_t)kFusedMaxM * (size_t)d * 4);
+  L.zero_end = off;
   L.a = off;
   off += align256((size_t)M * (size_t)I * 2);
-  L.acc = off;
-  off += align256((size_t)(M < 4 ? M : 4) * (size_t)d * 4);
-  if (M > 4) {
+  if (M > kFusedMaxM && tc_supported(M, d, I, 16)) {  // the tensor-core path may run
     const TcSizes z = tc_sizes(M, d, I, kTcMaxCtas);
     L.b_hl = off;
     off += align256(z.b_hl);
@@ -116,6 +120,7 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
     L.partials = off;
     off += align256(z.partials);
     L.counters = off;
+    L.ncounters = z.counters / 4;
     off += align256(z.counters);
   }
   L.total = off;
@@ -221,11 +226,13 @@ fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t
   st = device_for_launch(&dev);
   if (st != FMLP_OK) return st;
   cudaError_t e;
-  if (use_tc(M, d, I, 16))
-    e = launch_tc_down(a, M, W_down, d, I, residual, out,
-                       tc_workspace(workspace, workspace_layout(M, d, I)), *dev,
-                       (cudaStream_t)stream);
-  else
+  if (use_tc(M, d, I, 16)) {
+    // Run alone, the down GEMM has no prologue to clear its arrival counters.
+    const TcWorkspace tw = tc_workspace(workspace, workspace_layout(M, d, I));
+    e = cudaMemsetAsync(tw.counters, 0, (size_t)tw.ncounters * 4, (cudaStream_t)stream);
+    if (e == cudaSuccess)
+      e = launch_tc_down(a, M, W_down, d, I, residual, out, tw, *dev, (cudaStream_t)stream);
+  } else
     e = launch_down_stream(a, M, W_down, d, I, residual, out, status_word(workspace), *dev,
                            (cudaStream_t)stream);
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);

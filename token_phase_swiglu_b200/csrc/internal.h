@@ -21,17 +21,21 @@ cudaError_t current_device_info(const DeviceInfo** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 // The first 256 bytes are control words: the device status word at 0 and the
-// fused kernel's finished-CTA counter at 128.  Then the bf16 intermediate a
-// [M x I] (two-kernel path) and the fused kernel's f32 accumulator [M x d]
-// (M <= 4); the counter and the accumulator return to zero after every call.
+// fused kernel's finished-CTA counter at 128.  Everything below `zero_end` must read zero when a call
+// starts and is left at zero by every call (acc by the fused kernel's last
+// CTA, also after a timeout); its extent depends on d only, so one workspace
+// serves calls of any M and I at a fixed d.
 struct WorkspaceLayout {
   size_t status = 0;     // uint32 device status word
   size_t done = 128;     // uint32 finished-CTA counter (fused kernel)
+  size_t acc = 0;        // f32 [kFusedMaxM x d] accumulator (fused kernel)
+  size_t zero_end = 0;
   size_t a = 0;          // bf16 [M x I] intermediate
-  size_t acc = 0;        // f32 [min(M,4) x d] accumulator (fused kernel)
-  size_t b_hl = 0, rinv = 0, partials = 0, counters = 0;  // tensor-core path (M > 4)
+  size_t b_hl = 0, rinv = 0, partials = 0, counters = 0;  // tensor-core path
+  size_t ncounters = 0;
   size_t total = 0;
 };
+constexpr int kFusedMaxM = 4;  // token rows handled by the fused decode kernel
 WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I);
 
 constexpr uint32_t kStatusTimeout = 1u;
@@ -73,7 +77,8 @@ struct TcWorkspace {
   void* b_hl;          // bf16 token-tiled [hi; lo] rows of x*gamma
   float* rinv;         // [M] 1/RMS
   float* partials;     // stream-K partial accumulators
-  uint32_t* counters;  // per-tile arrival counters (zero between calls)
+  uint32_t* counters;  // per-tile arrival counters (zeroed by the prologue)
+  int ncounters;
   uint32_t* status;
 };
 struct TcSizes {

@@ -933,7 +933,7 @@ struct FusedPlan {
 // 256 columns per CTA, and a ring of at least three stages.
 FusedPlan make_fused_plan(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev) {
   FusedPlan f;
-  if (M < 1 || M > 4) return f;
+  if (M < 1 || M > kFusedMaxM) return f;
   const size_t budget = (size_t)dev.max_smem_optin - 1024;
   f.units = (int)(I / 8);
   f.grid = std::min(f.units, dev.sm_count);

@@ -98,18 +98,42 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
-// 32 lanes x 8 consecutive 32-bit columns; thread i of the warp gets lane
-// (32 * (warp % 4) + i), columns col..col+7.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
+// 32 lanes x W consecutive 32-bit columns (W = 8, 16, 32); thread i of the
+// warp gets lane (32 * (warp % 4) + i), columns col..col+W-1.  No wait:
+// several loads may be in flight; tmem_wait() before using the values.
+template <int W>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[W]);
+template <>
+__device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Barrier of the four epilogue warps that also ORs a failure flag, so that a
@@ -174,8 +198,9 @@ struct TcParams {
   int rows;            // valid A rows (2I packed rows, or d)
   int T;               // interleave tile (SwiGLU)
   int I, d;
-  int stages, stage_bytes, b_bytes;
-  uint32_t tmem_cols;  // allocated TMEM columns (2 x N rounded up to a power of two)
+  int C;               // accumulator chains per tile: MMA k-slice j goes to chain j % C
+  int stages, stage_bytes, a_bytes, b_bytes;
+  uint32_t tmem_cols;  // allocated TMEM columns (2 x C x N rounded up to a power of two)
   const float* rinv;   // [M] 1/RMS per token (SwiGLU)
   __nv_bfloat16* a_out;             // SwiGLU output a [M x I]
   float* out;                       // down output [M x d]
@@ -207,10 +232,8 @@ __device__ __forceinline__ void tc_flag(TcShared* sh, uint32_t* status) {
 // Epilogue of CW logical columns [col0, col0 + CW) of one finished tile
 // (warps 2-5; vals[j] = D[row, col0 + j], hi + lo already summed).
 template <int CW>
-__device__ __forceinline__ void epilogue_columns(const TcParams& p, int tile, const float (&vals)[CW],
-                                                 int col0, int r_local) {
-  const int rt = tile / p.sched.ntok, tt = tile % p.sched.ntok;
-  const int row = rt * kBM + r_local;
+__device__ __forceinline__ void epilogue_columns(const TcParams& p, int tt, int row,
+                                                 const float (&vals)[CW], int col0) {
   if (p.epi == kEpiDown) {
     const int n = row;
 #pragma unroll
@@ -252,25 +275,38 @@ __device__ __forceinline__ void epilogue_columns(const TcParams& p, int tile, co
   }
 }
 
-// Finish one tile: sum the accumulator (hi + lo for SwiGLU) with the other
-// contributors' partials, CW logical columns at a time.
+// Load CW columns at `col` of the tile's accumulator: the sum of its C chains.
+template <int CW>
+__device__ __forceinline__ void tile_cols(const TcParams& p, uint32_t tb, int col, float (&v)[CW]) {
+  uint32_t r[CW];
+  tmem_ld<CW>(tb + col, r);
+  tmem_wait();
+#pragma unroll
+  for (int j = 0; j < CW; ++j) v[j] = __uint_as_float(r[j]);
+  for (int c = 1; c < p.C; ++c) {
+    tmem_ld<CW>(tb + (uint32_t)(c * p.N) + col, r);
+    tmem_wait();
+#pragma unroll
+    for (int j = 0; j < CW; ++j) v[j] += __uint_as_float(r[j]);
+  }
+}
+
+// Finish a tile: its accumulator (hi + lo for SwiGLU) plus the other
+// contributors' partials, CW logical columns at a time, then the epilogue.
 template <int CW>
 __device__ void finish_tile(const TcParams& p, int t, uint32_t tb, bool whole, int c_first,
                             int c_last, int r_local) {
   const int ncol = p.epi == kEpiSwiGLU ? p.Mt : p.N;
+  const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
+  const int row = rt * kBM + r_local;
   for (int c0 = 0; c0 < ncol; c0 += CW) {
     float vals[CW];
+    tile_cols<CW>(p, tb, c0, vals);
+    if (p.epi == kEpiSwiGLU) {
+      float lo[CW];
+      tile_cols<CW>(p, tb, p.Mt + c0, lo);  // lo half of x*gamma
 #pragma unroll
-    for (int c = 0; c < CW; c += 8) {
-      float v[8];
-      tmem_ld8(tb + c0 + c, v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) vals[c + j] = v[j];
-      if (p.epi == kEpiSwiGLU) {
-        tmem_ld8(tb + p.Mt + c0 + c, v);  // lo half of x*gamma
-#pragma unroll
-        for (int j = 0; j < 8; ++j) vals[c + j] += v[j];
-      }
+      for (int j = 0; j < CW; ++j) vals[j] += lo[j];
     }
     if (!whole) {
       for (int cc = c_first; cc <= c_last; ++cc) {
@@ -286,7 +322,7 @@ __device__ void finish_tile(const TcParams& p, int t, uint32_t tb, bool whole, i
         }
       }
     }
-    epilogue_columns<CW>(p, t, vals, c0, r_local);
+    epilogue_columns<CW>(p, tt, row, vals, c0);
   }
 }
 
@@ -356,13 +392,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
           }
           const int slot = k % p.stages;
           uint8_t* a_dst = stage0 + (size_t)slot * p.stage_bytes;
-          uint8_t* b_dst = a_dst + kATileBytes;
+          uint8_t* b_dst = a_dst + p.a_bytes;
           if (k >= p.stages) {
             if (k == p.stages) {
               // activations of the early stages, now that they are written
               grid_dependency_wait();
               for (int e = 0; e < n_early; ++e)
-                tma_load_2d(stage0 + (size_t)e * p.stage_bytes + kATileBytes, &p.b_map,
+                tma_load_2d(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map,
                             early_kb[e] * kBK, early_tt[e] * brow_mul, &sh.full[e], pol_b);
             }
             if (!mbar_wait_bounded(&sh.empty[slot], (uint32_t)(((k / p.stages) - 1) & 1),
@@ -372,7 +408,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
               break;
             }
           }
-          mbar_arrive_expect_tx(&sh.full[slot], (uint32_t)(kATileBytes + p.b_bytes));
+          mbar_arrive_expect_tx(&sh.full[slot], (uint32_t)(p.a_bytes + p.b_bytes));
           tma_load_2d(a_dst, &p.a_map, kb * kBK, rt * kBM, &sh.full[slot], pol_a);
           if (k < p.stages) {
             early_kb[k] = kb;
@@ -387,7 +423,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
         // the whole range fit in the first ring: its activations are still owed
         grid_dependency_wait();
         for (int e = 0; e < k; ++e)
-          tma_load_2d(stage0 + (size_t)e * p.stage_bytes + kATileBytes, &p.b_map,
+          tma_load_2d(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map,
                       early_kb[e] * kBK, early_tt[e] * brow_mul, &sh.full[e], pol_b);
       }
     }
@@ -409,7 +445,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(buf * p.N);
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * p.C * p.N);
         for (int kb = kb0; kb < kb1; ++kb, ++k) {
           const int slot = k % p.stages;
           if (!mbar_wait_bounded(&sh.full[slot], (uint32_t)((k / p.stages) & 1), p.wait_ns,
@@ -420,11 +456,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stage0 + (size_t)slot * p.stage_bytes);
-          const uint32_t b_addr = a_addr + kATileBytes;
+          const uint32_t b_addr = a_addr + p.a_bytes;
+          // k-slice kk accumulates into chain kk % C: C independent MMA chains
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            mma_bf16(d_tmem, sw128_desc(a_addr + kk * 32), sw128_desc(b_addr + kk * 32), idesc,
-                     (kb > kb0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const int c = kk % p.C;
+            mma_bf16(d_tmem + (uint32_t)(c * p.N), sw128_desc(a_addr + kk * 32),
+                     sw128_desc(b_addr + kk * 32), idesc, (kb > kb0 || kk >= p.C) ? 1u : 0u);
+          }
           mma_commit(&sh.empty[slot]);  // stage reusable once these MMAs finish
         }
         if (ok) mma_commit(&sh.acc_full[buf]);
@@ -450,20 +489,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
       if (!got && lane == 0) tc_flag(&sh, p.status);
       if (epilogue_barrier_any(!got)) break;
       tc_fence_after();
-      const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.N);
+      const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.C * p.N);
       const bool whole = kb0 == 0 && kb1 == p.sched.KB;
       const int c_first = p.sched.cta_of((int64_t)t * p.sched.KB);
       const int c_last = p.sched.cta_of((int64_t)t * p.sched.KB + p.sched.KB - 1);
       bool finalize = whole;
       if (!whole) {
-        // this CTA's partial: slot 0 if the tile is where its range starts, else 1
+        // this CTA's partial (chains summed): slot 0 if the tile is where its
+        // range starts, else 1.  N is a multiple of 16.
         const int slot = (t == (int)(u0 / p.sched.KB)) ? 0 : 1;
         float* part = p.partials + ((size_t)blockIdx.x * 2 + slot) * (size_t)p.N * kBM;
-        for (int c = 0; c < p.N; c += 8) {
-          float v[8];
-          tmem_ld8(tb + c, v);
+        int c = 0;
+        for (; c + 32 <= p.N; c += 32) {
+          float v[32];
+          tile_cols<32>(p, tb, c, v);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) __stcg(part + (size_t)(c + j) * kBM + r_local, v[j]);
+          for (int j = 0; j < 32; ++j) __stcg(part + (size_t)(c + j) * kBM + r_local, v[j]);
+        }
+        if (c < p.N) {
+          float v[16];
+          tile_cols<16>(p, tb, c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(part + (size_t)(c + j) * kBM + r_local, v[j]);
         }
         __threadfence();
         named_barrier_sync(1, 128);
@@ -473,8 +520,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
         if (finalize) __threadfence();
       }
       if (finalize) {
-        if (ncol >= 32) finish_tile<32>(p, t, tb, whole, c_first, c_last, r_local);
-        else if (ncol >= 16) finish_tile<16>(p, t, tb, whole, c_first, c_last, r_local);
+        // a chunk width that divides the logical columns (a multiple of 8)
+        if (ncol % 32 == 0) finish_tile<32>(p, t, tb, whole, c_first, c_last, r_local);
+        else if (ncol % 16 == 0) finish_tile<16>(p, t, tb, whole, c_first, c_last, r_local);
         else finish_tile<8>(p, t, tb, whole, c_first, c_last, r_local);
         if (!whole && et == 0) atomicExch(p.counters + t, 0u);
       }
@@ -504,9 +552,16 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
                                                  const __nv_bfloat16* __restrict__ gamma,
                                                  float eps, int M, int d, int Mt,
                                                  __nv_bfloat16* __restrict__ b_hl,
-                                                 float* __restrict__ rinv) {
+                                                 float* __restrict__ rinv,
+                                                 uint32_t* __restrict__ counters,
+                                                 int ncounters) {
   grid_dependency_wait();
   grid_launch_dependents();
+  // The stream-K arrival counters start every call at zero, whatever a
+  // previous call (an aborted one, or one of another shape) left there.  The
+  // previous call's kernels are complete once the wait above returns.
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < ncounters; i += gridDim.x * blockDim.x)
+    counters[i] = 0u;
   const int slot = blockIdx.x;
   const int j = slot / Mt, i = slot % Mt;
   const int m = slot;
@@ -549,10 +604,11 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
 // Host side
 // ---------------------------------------------------------------------------
 struct TcPlan {
-  int N = 0, Mt = 0, ntok = 0, stages = 0, stage_bytes = 0, b_bytes = 0;
+  int N = 0, Mt = 0, ntok = 0, C = 0, stages = 0, stage_bytes = 0, a_bytes = 0, b_bytes = 0;
   uint32_t tmem_cols = 0;
   size_t smem = 0;
 };
+
 
 uint32_t pow2_at_least(uint32_t n) {
   uint32_t c = 32;
@@ -560,22 +616,30 @@ uint32_t pow2_at_least(uint32_t n) {
   return c;
 }
 
+// Tile shape of one GEMM: token tile Mt (N = 2 Mt for the hi/lo gate-up
+// operand) and C accumulator chains (2 C N TMEM columns <= 512, double-buffered).
+void tc_shape(int epi, int64_t M, int& Mt, int& N, int& C) {
+  if (epi == kEpiSwiGLU) {
+    Mt = (int)std::min<int64_t>(128, (M + 7) / 8 * 8);
+    N = 2 * Mt;
+  } else {
+    Mt = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
+    N = Mt;
+  }
+  C = 4 * N <= 256 ? 4 : (2 * N <= 256 ? 2 : 1);
+}
+
 TcPlan make_tc_plan(int epi, int64_t M, const DeviceInfo& dev) {
   TcPlan pl;
-  if (epi == kEpiSwiGLU) {
-    pl.Mt = (int)std::min<int64_t>(128, (M + 7) / 8 * 8);
-    pl.N = 2 * pl.Mt;
-  } else {
-    pl.Mt = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
-    pl.N = pl.Mt;
-  }
+  tc_shape(epi, M, pl.Mt, pl.N, pl.C);
   pl.ntok = (int)((M + pl.Mt - 1) / pl.Mt);
+  pl.a_bytes = kATileBytes;
   pl.b_bytes = pl.N * kBK * 2;
-  pl.stage_bytes = (kATileBytes + pl.b_bytes + 1023) / 1024 * 1024;
+  pl.stage_bytes = (pl.a_bytes + pl.b_bytes + 1023) / 1024 * 1024;
   const size_t budget = (size_t)dev.max_smem_optin - 2048 - 1024;  // static + alignment slack
   pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
   pl.smem = (size_t)pl.stages * pl.stage_bytes + 1024;
-  pl.tmem_cols = pow2_at_least((uint32_t)(2 * pl.N));
+  pl.tmem_cols = pow2_at_least((uint32_t)(2 * pl.C * pl.N));
   return pl;
 }
 
@@ -617,8 +681,10 @@ void fill_common(TcParams& p, const TcPlan& pl, int epi, int64_t M, int rows, in
   p.Mt = pl.Mt;
   p.M = (int)M;
   p.rows = rows;
+  p.C = pl.C;
   p.stages = pl.stages;
   p.stage_bytes = pl.stage_bytes;
+  p.a_bytes = pl.a_bytes;
   p.b_bytes = pl.b_bytes;
   p.tmem_cols = pl.tmem_cols;
   p.sched.KB = (K + kBK - 1) / kBK;
@@ -638,15 +704,15 @@ void fill_common(TcParams& p, const TcPlan& pl, int epi, int64_t M, int rows, in
 TcSizes tc_sizes(int64_t M, int64_t d, int64_t I, int sm_count) {
   if (M < 1) return TcSizes();
   TcSizes z;
-  const int Mt_g = (int)std::min<int64_t>(128, (M + 7) / 8 * 8);
-  const int ntok_g = (int)((M + Mt_g - 1) / Mt_g);
+  int Mt_g, N_g, C_g, Mt_d, N_d, C_d;
+  tc_shape(kEpiSwiGLU, M, Mt_g, N_g, C_g);
+  tc_shape(kEpiDown, M, Mt_d, N_d, C_d);
+  const int64_t ntok_g = (M + Mt_g - 1) / Mt_g, ntok_d = (M + Mt_d - 1) / Mt_d;
   z.b_hl = (size_t)ntok_g * 2 * Mt_g * d * 2;
   z.rinv = (size_t)M * 4;
-  const int N_max = std::max(2 * Mt_g, (int)std::min<int64_t>(256, (M + 15) / 16 * 16));
-  z.partials = (size_t)sm_count * 2 * N_max * kBM * 4;
+  z.partials = (size_t)sm_count * 2 * std::max(N_g, N_d) * kBM * 4;
   const int64_t tiles_g = ((2 * I + kBM - 1) / kBM) * ntok_g;
-  const int Mt_d = (int)std::min<int64_t>(256, (M + 15) / 16 * 16);
-  const int64_t tiles_d = ((d + kBM - 1) / kBM) * ((M + Mt_d - 1) / Mt_d);
+  const int64_t tiles_d = ((d + kBM - 1) / kBM) * ntok_d;
   z.counters = (size_t)std::max(tiles_g, tiles_d) * 4;
   return z;
 }
@@ -672,7 +738,8 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, act_split, (const __nv_bfloat16*)x,
                                        (const __nv_bfloat16*)gamma, eps, (int)M, (int)d, pl.Mt,
-                                       (__nv_bfloat16*)ws.b_hl, ws.rinv);
+                                       (__nv_bfloat16*)ws.b_hl, ws.rinv, ws.counters,
+                                       ws.ncounters);
     if (e != cudaSuccess) return e;
     note_launches(1);
   }
