@@ -80,12 +80,11 @@ FMLP_API fmlp_status fmlp_pack(const void* W_gate, const void* W_up, int64_t d, 
 /*
  * fmlp_workspace_bytes -- bytes of device workspace fmlp_forward needs for
  * (M, d, I).  The workspace holds a device status word, the fused decode
- * kernel's completion counter and f32 accumulator, the bf16 intermediate
- * a [M x I], and the tensor-core path's operand copy and stream-K partials.
- * A workspace must be zero-filled before its first use and again before it
- * serves a call with a larger d than all calls before; in between, every
- * call (a timed-out one too) leaves it ready for the next call of any M and
- * I.  Returns 0 for invalid sizes.
+ * kernel's two completion counters, the bf16 intermediate a [M x I], and
+ * the tensor-core path's operand copy and stream-K partials.  A workspace
+ * must be zero-filled before its first use; after that, every call (a
+ * timed-out one too) leaves it ready for the next call of any sizes whose
+ * fmlp_workspace_bytes it does not exceed.  Returns 0 for invalid sizes.
  */
 FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
 

@@ -104,10 +104,9 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
   WorkspaceLayout L;
   size_t off = 0;
   L.status = off;
+  L.inited = off + 64;
   L.done = off + 128;
   off += 256;
-  L.acc = off;
-  off += align256((size_t)kFusedMaxM * (size_t)d * 4);
   L.zero_end = off;
   L.a = off;
   off += align256((size_t)M * (size_t)I * 2);
@@ -260,10 +259,10 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   if (fused_decode_supported(M, d, I, *dev)) {
-    float* acc = (float*)((char*)workspace + L.acc);
+    uint32_t* inited = (uint32_t*)((char*)workspace + L.inited);
     uint32_t* done = (uint32_t*)((char*)workspace + L.done);
-    e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out, acc,
-                            done, status, *dev, s);
+    e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out,
+                            inited, done, status, *dev, s);
   } else if (use_tc(M, d, I, tile_T)) {
     const TcWorkspace tw = tc_workspace(workspace, L);
     e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, tw, *dev, s);

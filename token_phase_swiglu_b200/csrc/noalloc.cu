@@ -78,9 +78,9 @@ extern "C" fmlp_status fmlp_forward_noalloc(const void* x, int64_t M, const void
   cudaError_t e = scratch_on_current_device(&scratch);
   if (e != cudaSuccess) return fmlp::record_cuda_error(e);
   if (M > 0) {
-    // The buffer keeps whatever the previous call left, possibly for another
-    // d.  The status word, the fused kernel's counter and its accumulator must
-    // start at zero; every other region is rewritten before it is read.
+    // The buffer keeps whatever the previous call left.  The control words
+    // (status word and the fused kernel's counters) must start at zero; every
+    // other region is rewritten before it is read.
     const size_t zero_bytes = fmlp::workspace_layout(M, d, I).zero_end;
     e = cudaMemsetAsync(scratch, 0, zero_bytes, (cudaStream_t)stream);
     if (e != cudaSuccess) return fmlp::record_cuda_error(e);

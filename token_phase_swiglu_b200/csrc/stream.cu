@@ -267,8 +267,22 @@ __device__ bool produce_gateup(Producer& pr, const GateUpGeom& g, int g0, int n_
   return true;
 }
 
+// gamma (weights: ready before the previous kernel ends) as f32 in row 0 of
+// s, in the layout stage_x_gamma uses; consumer threads, before the
+// dependency wait.  Each thread touches only the vectors it handles later.
+__device__ void stage_gamma(const __nv_bfloat16* gamma, int d, float* s) {
+  const int ct = threadIdx.x - 32;
+  for (int v = ct; v < d / 8; v += kConsumers * 32) {
+    const uint4 gv = ld_keep(gamma + (int64_t)v * 8);
+    float4* dst = reinterpret_cast<float4*>(s);
+    dst[v] = make_float4(bf16lo(gv.x), bf16hi(gv.x), bf16lo(gv.y), bf16hi(gv.y));
+    dst[d / 8 + v] = make_float4(bf16lo(gv.z), bf16hi(gv.z), bf16lo(gv.w), bf16hi(gv.w));
+  }
+}
+
 // s = x * gamma (exact in f32) for the CTA's token rows, and r = 1/sqrt(mean x^2 + eps).
 // Row m of s holds d/8 float4 of columns 8v..8v+3, then d/8 float4 of 8v+4..8v+7.
+// If `gamma` is null, row 0 of s already holds gamma (stage_gamma).
 template <int MT>
 __device__ void stage_x_gamma(const __nv_bfloat16* x, const __nv_bfloat16* gamma, float eps,
                               int d, int m0, int mt, float* s, float (*red)[MT], float* rinv) {
@@ -277,15 +291,27 @@ __device__ void stage_x_gamma(const __nv_bfloat16* x, const __nv_bfloat16* gamma
 #pragma unroll
   for (int m = 0; m < MT; ++m) ss[m] = 0.f;
   for (int v = ct; v < d / 8; v += kConsumers * 32) {
-    const uint4 gv = ld_keep(gamma + (int64_t)v * 8);
-    const float gf[8] = {bf16lo(gv.x), bf16hi(gv.x), bf16lo(gv.y), bf16hi(gv.y),
-                         bf16lo(gv.z), bf16hi(gv.z), bf16lo(gv.w), bf16hi(gv.w)};
+    float gf[8];
+    if (gamma) {
+      const uint4 gv = ld_keep(gamma + (int64_t)v * 8);
+      gf[0] = bf16lo(gv.x); gf[1] = bf16hi(gv.x); gf[2] = bf16lo(gv.y); gf[3] = bf16hi(gv.y);
+      gf[4] = bf16lo(gv.z); gf[5] = bf16hi(gv.z); gf[6] = bf16lo(gv.w); gf[7] = bf16hi(gv.w);
+    } else {
+      const float4 g0 = reinterpret_cast<const float4*>(s)[v];
+      const float4 g1 = reinterpret_cast<const float4*>(s)[d / 8 + v];
+      gf[0] = g0.x; gf[1] = g0.y; gf[2] = g0.z; gf[3] = g0.w;
+      gf[4] = g1.x; gf[5] = g1.y; gf[6] = g1.z; gf[7] = g1.w;
+    }
+    uint4 xv[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {  // all loads first: one L2 round trip
+      xv[m] = make_uint4(0, 0, 0, 0);
+      if (m < mt) xv[m] = ld_keep(x + (int64_t)(m0 + m) * d + (int64_t)v * 8);
+    }
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      uint4 xv = make_uint4(0, 0, 0, 0);
-      if (m < mt) xv = ld_keep(x + (int64_t)(m0 + m) * d + (int64_t)v * 8);
-      const float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
-                           bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+      const float xf[8] = {bf16lo(xv[m].x), bf16hi(xv[m].x), bf16lo(xv[m].y), bf16hi(xv[m].y),
+                           bf16lo(xv[m].z), bf16hi(xv[m].z), bf16lo(xv[m].w), bf16hi(xv[m].w)};
 #pragma unroll
       for (int e = 0; e < 8; ++e) ss[m] = fmaf(xf[e], xf[e], ss[m]);
       // two planes of float4 (columns 8v..8v+3, then 8v+4..8v+7) so that lanes
@@ -549,12 +575,13 @@ __device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_by
     }
     __syncwarp();
   } else {
+    if (GATE) stage_gamma(p.gamma, p.gu.d, reinterpret_cast<float*>(act));
     grid_dependency_wait();  // inputs may be written by the previous kernel
     Consumer cs{ring, &st, p.ctl, 0, lane};
     bool ok = true;
     if (GATE) {
       float rinv[MT];
-      stage_x_gamma<MT>(p.x, p.gamma, p.eps, p.gu.d, m0, mt, reinterpret_cast<float*>(act),
+      stage_x_gamma<MT>(p.x, nullptr, p.eps, p.gu.d, m0, mt, reinterpret_cast<float*>(act),
                         red, rinv);
       ok = consume_gateup<MT>(cs, p.gu, ga0, nga, reinterpret_cast<const float*>(act), rinv,
                               p.a, m0, mt, xch);
@@ -586,8 +613,8 @@ struct FusedParams {
   const __nv_bfloat16* x;
   const __nv_bfloat16* gamma;
   const __nv_bfloat16* residual;
-  float* out;
-  float* acc;          // [M x d] f32 accumulator (zero between calls)
+  float* out;          // [M x d] f32: set to the residual (or 0), then CTAs add into it
+  uint32_t* inited;    // CTAs whose share of out is set (zero between calls)
   uint32_t* done;      // CTAs finished (zero between calls)
   Control ctl;
   GateUpGeom gu;
@@ -668,11 +695,44 @@ __device__ bool consume_down_slice(Consumer& cs, const FusedParams& p, const flo
       }
 #pragma unroll
       for (int m = 0; m < MT; ++m)
-        if (m < mt) atomicAdd(p.acc + (int64_t)m * p.d + n, acc[0][m] + acc[1][m]);
+        if (m < mt) atomicAdd(p.out + (int64_t)m * p.d + n, acc[0][m] + acc[1][m]);
     }
     cs.release();
   }
   return true;
+}
+
+// Wait (one thread) until the counter at `ctr` reaches `target`, with
+// acquire semantics, for at most limit_ns; false if it gave up.
+__device__ bool wait_counter(const uint32_t* ctr, uint32_t target, uint64_t limit_ns,
+                             volatile int* abort) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(32);
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (abort && *abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Warp 0, lanes 1-31: this CTA's share of out (float4 granules) set to the
+// residual or to zero, then counted in `inited`.
+__device__ void init_out_share(const FusedParams& p, int mt, int lane) {
+  grid_dependency_wait();  // out and the residual belong to the stream's order
+  const int64_t n4 = (int64_t)mt * p.d / 4;
+  const int64_t q0 = n4 * blockIdx.x / gridDim.x, q1 = n4 * (blockIdx.x + 1) / gridDim.x;
+  for (int64_t i = q0 + lane - 1; i < q1; i += 31) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p.residual) {
+      const uint2 r = __ldg(reinterpret_cast<const uint2*>(p.residual) + i);
+      v = make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+    }
+    reinterpret_cast<float4*>(p.out)[i] = v;
+  }
+  __threadfence();
+  __syncwarp(0xfffffffeu);
+  if (lane == 1) atomicAdd(p.inited, 1u);
 }
 
 template <int MT>
@@ -681,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
   __shared__ float red[kConsumers][MT];
   __shared__ float xch[2 * kGroup * 2 * MT];
   __shared__ CtaState st;
-  __shared__ int last_cta;
+  __shared__ int go;
 
   Ring ring;
   ring.full = reinterpret_cast<uint64_t*>(smem);
@@ -709,59 +769,46 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
       Producer pr{ring, &st, p.ctl, evict_first_policy(), ng * p.gu.nchunks + p.nrb};
       if (produce_gateup(pr, p.gu, g0, ng)) produce_down_slice(pr, p, i0);
       st.issued = pr.k;
+    } else {
+      init_out_share(p, mt, lane);
     }
     __syncwarp();
   } else {
-    grid_dependency_wait();  // inputs may be written by the previous kernel
     const int ct = threadIdx.x - 32;
+    stage_gamma(p.gamma, p.d, s);  // weights: before the dependency wait
+    grid_dependency_wait();        // x may be written by the previous kernel
     Consumer cs{ring, &st, p.ctl, 0, lane};
     float rinv[MT];
-    stage_x_gamma<MT>(p.x, p.gamma, p.eps, p.d, 0, mt, s, red, rinv);
-    bool ok = consume_gateup<MT>(cs, p.gu, g0, ng, s, rinv, nullptr, 0, mt, xch, slice, i0,
-                                 p.swbox);
-    named_barrier_sync(kBarStage, kConsumers * 32);  // the CTA's slice of a is complete
-    if (ok) consume_down_slice<MT>(cs, p, slice, w, mt);
-    // Completion count, also after a timeout, so that the last CTA always
-    // leaves acc and the counter at zero for the next call.
-    __threadfence();
-    named_barrier_sync(kBarStage, kConsumers * 32);
-    if (ct == 0) last_cta = atomicAdd(p.done, 1u) == gridDim.x - 1;
-    named_barrier_sync(kBarStage, kConsumers * 32);
-    if (last_cta) {
-      // out = acc (+ residual); acc back to zero.  d % 8 == 0, so float4 and
-      // four-element residual reads tile every row; all loads are issued
-      // before the stores to pay the L2 latency once.
-      __threadfence();
-      constexpr int kBatch = 8;
-      const int n4 = mt * p.d / 4;
-      for (int base = ct; base < n4; base += kConsumers * 32 * kBatch) {
-        float4 v[kBatch];
-        uint2 r[kBatch];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-          const int i = base + b * kConsumers * 32;
-          if (i < n4) {
-            v[b] = __ldcg(reinterpret_cast<const float4*>(p.acc) + i);
-            r[b] = p.residual ? __ldg(reinterpret_cast<const uint2*>(p.residual) + i)
-                              : make_uint2(0, 0);
-          }
-        }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-          const int i = base + b * kConsumers * 32;
-          if (i < n4) {
-            __stcg(reinterpret_cast<float4*>(p.acc) + i, make_float4(0.f, 0.f, 0.f, 0.f));
-            reinterpret_cast<float4*>(p.out)[i] =
-                make_float4(v[b].x + bf16lo(r[b].x), v[b].y + bf16hi(r[b].x),
-                            v[b].z + bf16lo(r[b].y), v[b].w + bf16hi(r[b].y));
-          }
-        }
+    stage_x_gamma<MT>(p.x, nullptr, p.eps, p.d, 0, mt, s, red, rinv);
+    const bool ok = consume_gateup<MT>(cs, p.gu, g0, ng, s, rinv, nullptr, 0, mt, xch, slice,
+                                       i0, p.swbox);
+    // Every CTA's share of out must be set before anyone adds into it.  The
+    // shares are written at the start, so by the end of the gate-up phase
+    // this normally returns at once (the ring keeps filling meanwhile).  The
+    // decision is published before the barrier so all consumer warps take it.
+    if (ct == 0) {
+      bool g = ok;
+      if (g && !wait_counter(p.inited, gridDim.x, p.ctl.wait_ns, &st.abort)) {
+        flag_timeout(&st, p.ctl.status);
+        g = false;
       }
-      if (ct == 0) atomicExch(p.done, 0u);
+      __threadfence();
+      go = g;
     }
+    named_barrier_sync(kBarStage, kConsumers * 32);  // slice of a complete, out ready
+    if (go) consume_down_slice<MT>(cs, p, slice, w, mt);
   }
   __syncthreads();
-  if (threadIdx.x == 0 && st.abort) drain_ring(ring, st.issued);
+  if (threadIdx.x == 0) {
+    if (st.abort) drain_ring(ring, st.issued);
+    // Every CTA has counted itself in `inited` and is past its wait on it:
+    // the last one to get here leaves both counters at zero for the next call
+    // (also after a timeout).
+    if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+      atomicExch(p.inited, 0u);
+      atomicExch(p.done, 0u);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -990,8 +1037,9 @@ bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& d
 
 cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                                const void* residual, float* out, float* acc, uint32_t* done,
-                                uint32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
+                                const void* residual, float* out, uint32_t* inited,
+                                uint32_t* done, uint32_t* status, const DeviceInfo& dev,
+                                cudaStream_t stream) {
   const FusedPlan f = make_fused_plan(M, d, I, dev);
   if (f.mt == 0) return cudaErrorInvalidConfiguration;
   FusedParams p;
@@ -1004,7 +1052,7 @@ cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, flo
   p.gamma = (const __nv_bfloat16*)gamma;
   p.residual = (const __nv_bfloat16*)residual;
   p.out = out;
-  p.acc = acc;
+  p.inited = inited;
   p.done = done;
   p.ctl.status = status;
   p.ctl.wait_ns = wait_timeout_ns();
