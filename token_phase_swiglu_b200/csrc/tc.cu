@@ -153,7 +153,7 @@ __device__ __forceinline__ bool epilogue_barrier_any(bool failed) {
 // Stream-K schedule
 // ---------------------------------------------------------------------------
 struct Sched {
-  int KB;      // k-blocks per tile
+  int KB;      // stages (groups of KS k-blocks) per tile
   int tiles;   // row tiles x token tiles
   int ntok;    // token tiles (tile index = row_tile * ntok + token_tile)
   int ctas;    // grid size
@@ -199,6 +199,8 @@ struct TcParams {
   int T;               // interleave tile (SwiGLU)
   int I, d;
   int C;               // accumulator chains per tile: MMA k-slice j goes to chain j % C
+  int KS;              // k-blocks per stage (one 3-D copy of A and one of B)
+  int KBtot;           // k-blocks of K
   int stages, stage_bytes, a_bytes, b_bytes;
   uint32_t tmem_cols;  // allocated TMEM columns (2 x C x N rounded up to a power of two)
   const float* rinv;   // [M] 1/RMS per token (SwiGLU)
@@ -398,8 +400,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
               // activations of the early stages, now that they are written
               grid_dependency_wait();
               for (int e = 0; e < n_early; ++e)
-                tma_load_2d(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map,
-                            early_kb[e] * kBK, early_tt[e] * brow_mul, &sh.full[e], pol_b);
+                tma_load_3d(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map, 0,
+                            early_tt[e] * brow_mul, early_kb[e] * p.KS, &sh.full[e], pol_b);
             }
             if (!mbar_wait_bounded(&sh.empty[slot], (uint32_t)(((k / p.stages) - 1) & 1),
                                    p.wait_ns, abort)) {
@@ -409,12 +411,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
             }
           }
           mbar_arrive_expect_tx(&sh.full[slot], (uint32_t)(p.a_bytes + p.b_bytes));
-          tma_load_2d(a_dst, &p.a_map, kb * kBK, rt * kBM, &sh.full[slot], pol_a);
+          tma_load_3d(a_dst, &p.a_map, 0, rt * kBM, kb * p.KS, &sh.full[slot], pol_a);
           if (k < p.stages) {
             early_kb[k] = kb;
             early_tt[k] = tt;
           } else {
-            tma_load_2d(b_dst, &p.b_map, kb * kBK, tt * brow_mul, &sh.full[slot], pol_b);
+            tma_load_3d(b_dst, &p.b_map, 0, tt * brow_mul, kb * p.KS, &sh.full[slot], pol_b);
           }
           sh.k_issued = k + 1;
         }
@@ -423,8 +425,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
         // the whole range fit in the first ring: its activations are still owed
         grid_dependency_wait();
         for (int e = 0; e < k; ++e)
-          tma_load_2d(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map,
-                      early_kb[e] * kBK, early_tt[e] * brow_mul, &sh.full[e], pol_b);
+          tma_load_3d(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map, 0,
+                      early_tt[e] * brow_mul, early_kb[e] * p.KS, &sh.full[e], pol_b);
       }
     }
     __syncwarp();
@@ -457,12 +459,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stage0 + (size_t)slot * p.stage_bytes);
           const uint32_t b_addr = a_addr + p.a_bytes;
-          // k-slice kk accumulates into chain kk % C: C independent MMA chains
+          const uint32_t b_kblock = (uint32_t)(p.N * kBK * 2);
+          // the last stage of K may hold fewer than KS k-blocks (the rest is zero fill)
+          const int nkb = min(p.KS, p.KBtot - kb * p.KS);
+          for (int kbi = 0; kbi < nkb; ++kbi) {
+            // k-slice kk accumulates into chain kk % C: C independent MMA chains
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const int c = kk % p.C;
-            mma_bf16(d_tmem + (uint32_t)(c * p.N), sw128_desc(a_addr + kk * 32),
-                     sw128_desc(b_addr + kk * 32), idesc, (kb > kb0 || kk >= p.C) ? 1u : 0u);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const int c = kk % p.C;
+              const bool first = kb == kb0 && kbi == 0 && kk < p.C;
+              mma_bf16(d_tmem + (uint32_t)(c * p.N),
+                       sw128_desc(a_addr + (uint32_t)(kbi * kATileBytes) + kk * 32),
+                       sw128_desc(b_addr + (uint32_t)kbi * b_kblock + kk * 32), idesc,
+                       first ? 0u : 1u);
+            }
           }
           mma_commit(&sh.empty[slot]);  // stage reusable once these MMAs finish
         }
@@ -604,7 +614,8 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
 // Host side
 // ---------------------------------------------------------------------------
 struct TcPlan {
-  int N = 0, Mt = 0, ntok = 0, C = 0, stages = 0, stage_bytes = 0, a_bytes = 0, b_bytes = 0;
+  int N = 0, Mt = 0, ntok = 0, C = 0, KS = 1, stages = 0, stage_bytes = 0, a_bytes = 0,
+      b_bytes = 0;
   uint32_t tmem_cols = 0;
   size_t smem = 0;
 };
@@ -629,15 +640,34 @@ void tc_shape(int epi, int64_t M, int& Mt, int& N, int& C) {
   C = 4 * N <= 256 ? 4 : (2 * N <= 256 ? 2 : 1);
 }
 
-TcPlan make_tc_plan(int epi, int64_t M, const DeviceInfo& dev) {
+#ifndef FMLP_TC_MAX_KS
+#define FMLP_TC_MAX_KS 4
+#endif
+#ifndef FMLP_TC_MIN_STAGES
+#define FMLP_TC_MIN_STAGES 2
+#endif
+
+// Stages of KS k-blocks.  On B200 one SM issues TMA copies at a few million
+// per second whatever their size (measured: ~2 M stages/s of two copies),
+// so a stage moves KS k-blocks of A and of B in one copy each, with KS as
+// large as still leaves FMLP_TC_MIN_STAGES stages: on the 8B-shaped decode
+// layers fewer, larger copies beat a deeper ring of small ones (M = 8:
+// 3.2 -> 5.0 TB/s).
+TcPlan make_tc_plan(int epi, int64_t M, int64_t K, const DeviceInfo& dev) {
   TcPlan pl;
   tc_shape(epi, M, pl.Mt, pl.N, pl.C);
   pl.ntok = (int)((M + pl.Mt - 1) / pl.Mt);
-  pl.a_bytes = kATileBytes;
-  pl.b_bytes = pl.N * kBK * 2;
-  pl.stage_bytes = (pl.a_bytes + pl.b_bytes + 1023) / 1024 * 1024;
   const size_t budget = (size_t)dev.max_smem_optin - 2048 - 1024;  // static + alignment slack
-  pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
+  const int kb_total = (int)(K / kBK);
+  for (int ks = FMLP_TC_MAX_KS; ks >= 1; ks /= 2) {
+    if (ks > 1 && ks > kb_total) continue;
+    pl.KS = ks;
+    pl.a_bytes = ks * kATileBytes;
+    pl.b_bytes = ks * pl.N * kBK * 2;
+    pl.stage_bytes = (pl.a_bytes + pl.b_bytes + 1023) / 1024 * 1024;
+    pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
+    if (pl.stages >= FMLP_TC_MIN_STAGES) break;
+  }
   pl.smem = (size_t)pl.stages * pl.stage_bytes + 1024;
   pl.tmem_cols = pow2_at_least((uint32_t)(2 * pl.C * pl.N));
   return pl;
@@ -682,12 +712,14 @@ void fill_common(TcParams& p, const TcPlan& pl, int epi, int64_t M, int rows, in
   p.M = (int)M;
   p.rows = rows;
   p.C = pl.C;
+  p.KS = pl.KS;
+  p.KBtot = K / kBK;
   p.stages = pl.stages;
   p.stage_bytes = pl.stage_bytes;
   p.a_bytes = pl.a_bytes;
   p.b_bytes = pl.b_bytes;
   p.tmem_cols = pl.tmem_cols;
-  p.sched.KB = (K + kBK - 1) / kBK;
+  p.sched.KB = (K / kBK + pl.KS - 1) / pl.KS;
   p.sched.ntok = pl.ntok;
   p.sched.tiles = ((rows + kBM - 1) / kBM) * pl.ntok;
   p.sched.ctas = (int)std::min<int64_t>(
@@ -724,7 +756,7 @@ bool tc_supported(int64_t M, int64_t d, int64_t I, int T) {
 cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float eps,
                              const void* P, int T, int64_t d, int64_t I, void* a,
                              const TcWorkspace& ws, const DeviceInfo& dev, cudaStream_t stream) {
-  const TcPlan pl = make_tc_plan(kEpiSwiGLU, M, dev);
+  const TcPlan pl = make_tc_plan(kEpiSwiGLU, M, d, dev);
   // prologue: hi/lo split of x * gamma into the token-tiled B operand, and 1/RMS
   {
     cudaLaunchConfig_t cfg = {};
@@ -746,11 +778,11 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
   TcParams p;
   memset(&p, 0, sizeof(p));
   const int rows = (int)(2 * I);
-  cudaError_t e = encode_tmap_2d_bf16(&p.a_map, P, (uint64_t)rows, (uint64_t)d, (uint64_t)d * 2,
-                                      kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+  cudaError_t e = encode_tmap_kblocks_bf16(&p.a_map, P, (uint64_t)rows, (uint64_t)d,
+                                           (uint64_t)d * 2, kBM, (uint32_t)pl.KS);
   if (e == cudaSuccess)
-    e = encode_tmap_2d_bf16(&p.b_map, ws.b_hl, (uint64_t)pl.ntok * 2 * pl.Mt, (uint64_t)d,
-                            (uint64_t)d * 2, (uint32_t)pl.N, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+    e = encode_tmap_kblocks_bf16(&p.b_map, ws.b_hl, (uint64_t)pl.ntok * 2 * pl.Mt, (uint64_t)d,
+                                 (uint64_t)d * 2, (uint32_t)pl.N, (uint32_t)pl.KS);
   if (e != cudaSuccess) return e;
   fill_common(p, pl, kEpiSwiGLU, M, rows, (int)d, ws, dev);
   p.T = T;
@@ -764,14 +796,14 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
 cudaError_t launch_tc_down(const void* a, int64_t M, const void* W_down, int64_t d, int64_t I,
                            const void* residual, float* out, const TcWorkspace& ws,
                            const DeviceInfo& dev, cudaStream_t stream) {
-  const TcPlan pl = make_tc_plan(kEpiDown, M, dev);
+  const TcPlan pl = make_tc_plan(kEpiDown, M, I, dev);
   TcParams p;
   memset(&p, 0, sizeof(p));
-  cudaError_t e = encode_tmap_2d_bf16(&p.a_map, W_down, (uint64_t)d, (uint64_t)I,
-                                      (uint64_t)I * 2, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+  cudaError_t e = encode_tmap_kblocks_bf16(&p.a_map, W_down, (uint64_t)d, (uint64_t)I,
+                                           (uint64_t)I * 2, kBM, (uint32_t)pl.KS);
   if (e == cudaSuccess)
-    e = encode_tmap_2d_bf16(&p.b_map, a, (uint64_t)M, (uint64_t)I, (uint64_t)I * 2,
-                            (uint32_t)pl.N, kBK, CU_TENSOR_MAP_SWIZZLE_128B);
+    e = encode_tmap_kblocks_bf16(&p.b_map, a, (uint64_t)M, (uint64_t)I, (uint64_t)I * 2,
+                                 (uint32_t)pl.N, (uint32_t)pl.KS);
   if (e != cudaSuccess) return e;
   fill_common(p, pl, kEpiDown, M, (int)d, (int)I, ws, dev);
   p.I = (int)I;

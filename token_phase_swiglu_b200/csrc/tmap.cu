@@ -45,4 +45,21 @@ cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t row
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_tmap_kblocks_bf16(CUtensorMap* map, const void* base, uint64_t rows,
+                                     uint64_t cols, uint64_t row_bytes, uint32_t box_rows,
+                                     uint32_t box_kblocks) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  cudaError_t e = encoder(&fn);
+  if (e != cudaSuccess) return e;
+  if (cols % 64 != 0) return cudaErrorInvalidValue;
+  const cuuint64_t dims[3] = {64, rows, cols / 64};
+  const cuuint64_t strides[2] = {row_bytes, 128};
+  const cuuint32_t box[3] = {64, box_rows, box_kblocks};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace fmlp
