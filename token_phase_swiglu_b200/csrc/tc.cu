@@ -150,15 +150,26 @@ __device__ __forceinline__ bool epilogue_barrier_any(bool failed) {
 }
 
 // ---------------------------------------------------------------------------
-// Stream-K schedule
+// Schedule: data-parallel rounds, then stream-K over the remainder.
+//
+// Tiles are numbered t = row_tile * ntok + token_tile.  In round r < dp
+// CTA c computes tile r * ctas + c whole, so the CTAs running at the same
+// time share each weight row tile across all token tiles and it crosses
+// HBM once (L2 serves the other token tiles).  The last one to two waves of
+// tiles are cut "stream-K": their (tile, stage) units are split evenly over
+// the CTAs, so a tile may be shared by a few CTAs; each writes its partial
+// accumulator to the workspace and the last one to arrive (tile counter)
+// sums them and runs the epilogue.
 // ---------------------------------------------------------------------------
 struct Sched {
   int KB;      // stages (groups of KS k-blocks) per tile
   int tiles;   // row tiles x token tiles
   int ntok;    // token tiles (tile index = row_tile * ntok + token_tile)
   int ctas;    // grid size
-  __device__ __forceinline__ int64_t units() const { return (int64_t)tiles * KB; }
-  // unit range of CTA c
+  int dp;      // data-parallel rounds (whole tiles per CTA)
+  __device__ __forceinline__ int sk_tile0() const { return dp * ctas; }
+  __device__ __forceinline__ int64_t units() const { return (int64_t)(tiles - sk_tile0()) * KB; }
+  // stream-K unit range of CTA c (units counted from the first stream-K tile)
   __device__ __forceinline__ void range(int c, int64_t& u0, int64_t& u1) const {
     const int64_t U = units(), per = U / ctas, rem = U % ctas;
     u0 = c * per + (c < rem ? (int64_t)c : rem);
@@ -169,16 +180,32 @@ struct Sched {
     const int64_t big = rem * (per + 1);
     return u < big ? (int)(u / (per + 1)) : (int)(rem + (u - big) / per);
   }
+  // first tile of CTA c's stream-K range
+  __device__ __forceinline__ int sk_first_tile(int c) const {
+    int64_t u0, u1;
+    range(c, u0, u1);
+    return sk_tile0() + (int)(u0 / KB);
+  }
 };
 
-// Segment s of this CTA's range: tile t, k-blocks [kb0, kb1).  Returns false past the end.
+// Segment s of this CTA's work: tile t, stages [kb0, kb1).  Segments
+// 0..dp-1 are the whole tiles of the data-parallel rounds; then the
+// stream-K range [u0, u1).  Returns false past the end.
 __device__ __forceinline__ bool segment(const Sched& S, int64_t u0, int64_t u1, int s, int& t,
                                         int& kb0, int& kb1) {
+  if (s < S.dp) {
+    t = s * S.ctas + (int)blockIdx.x;
+    kb0 = 0;
+    kb1 = S.KB;
+    return true;
+  }
+  s -= S.dp;
   if (u0 >= u1) return false;
   const int t0 = (int)(u0 / S.KB);
-  t = t0 + s;
-  const int64_t tb = (int64_t)t * S.KB;
+  const int tl = t0 + s;
+  const int64_t tb = (int64_t)tl * S.KB;
   if (tb >= u1) return false;
+  t = S.sk_tile0() + tl;
   kb0 = (int)(max(u0, tb) - tb);
   kb1 = (int)(min(u1, tb + S.KB) - tb);
   return true;
@@ -315,7 +342,7 @@ __device__ void finish_tile(const TcParams& p, int t, uint32_t tb, bool whole, i
         if (cc == (int)blockIdx.x) continue;
         int64_t cu0, cu1;
         p.sched.range(cc, cu0, cu1);
-        const int slot = (t == (int)(cu0 / p.sched.KB)) ? 0 : 1;
+        const int slot = (t == p.sched.sk_tile0() + (int)(cu0 / p.sched.KB)) ? 0 : 1;
         const float* part = p.partials + ((size_t)cc * 2 + slot) * (size_t)p.N * kBM;
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
@@ -501,13 +528,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
       tc_fence_after();
       const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.C * p.N);
       const bool whole = kb0 == 0 && kb1 == p.sched.KB;
-      const int c_first = p.sched.cta_of((int64_t)t * p.sched.KB);
-      const int c_last = p.sched.cta_of((int64_t)t * p.sched.KB + p.sched.KB - 1);
+      const int64_t tu = (int64_t)(t - p.sched.sk_tile0()) * p.sched.KB;  // stream-K tiles only
+      const int c_first = whole ? 0 : p.sched.cta_of(tu);
+      const int c_last = whole ? 0 : p.sched.cta_of(tu + p.sched.KB - 1);
       bool finalize = whole;
       if (!whole) {
         // this CTA's partial (chains summed): slot 0 if the tile is where its
         // range starts, else 1.  N is a multiple of 16.
-        const int slot = (t == (int)(u0 / p.sched.KB)) ? 0 : 1;
+        const int slot = (t == p.sched.sk_tile0() + (int)(u0 / p.sched.KB)) ? 0 : 1;
         float* part = p.partials + ((size_t)blockIdx.x * 2 + slot) * (size_t)p.N * kBM;
         int c = 0;
         for (; c + 32 <= p.N; c += 32) {
@@ -724,6 +752,12 @@ void fill_common(TcParams& p, const TcPlan& pl, int epi, int64_t M, int rows, in
   p.sched.tiles = ((rows + kBM - 1) / kBM) * pl.ntok;
   p.sched.ctas = (int)std::min<int64_t>(
       {(int64_t)p.sched.tiles * p.sched.KB, (int64_t)dev.sm_count, (int64_t)kTcMaxCtas});
+  // With one token tile no weight tile is reused, so plain stream-K balances
+  // best.  Otherwise whole waves run data-parallel, and the stream-K rest is
+  // kept at half a wave or more (folding one wave into it if needed) so that
+  // a stream-K tile has only a few contributors.
+  const int waves = p.sched.tiles / p.sched.ctas, rest = p.sched.tiles % p.sched.ctas;
+  p.sched.dp = pl.ntok == 1 ? 0 : (2 * rest >= p.sched.ctas ? waves : std::max(0, waves - 1));
   p.partials = ws.partials;
   p.counters = ws.counters;
   p.status = ws.status;
