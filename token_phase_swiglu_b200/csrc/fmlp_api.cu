@@ -202,7 +202,7 @@ fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* gamma, flo
   if (st != FMLP_OK) return st;
   cudaError_t e;
   if (use_tc(M, d, I, tile_T))
-    e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a,
+    e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, nullptr, nullptr,
                          tc_workspace(workspace, workspace_layout(M, d, I)), *dev,
                          (cudaStream_t)stream);
   else
@@ -226,11 +226,10 @@ fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t
   if (st != FMLP_OK) return st;
   cudaError_t e;
   if (use_tc(M, d, I, 16)) {
-    // Run alone, the down GEMM has no prologue to clear its arrival counters.
+    // Run alone, the down GEMM has no gate-up prologue to set out first.
     const TcWorkspace tw = tc_workspace(workspace, workspace_layout(M, d, I));
-    e = cudaMemsetAsync(tw.counters, 0, (size_t)tw.ncounters * 4, (cudaStream_t)stream);
-    if (e == cudaSuccess)
-      e = launch_tc_down(a, M, W_down, d, I, residual, out, tw, *dev, (cudaStream_t)stream);
+    e = launch_out_init(out, residual, M, d, *dev, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = launch_tc_down(a, M, W_down, d, I, out, tw, *dev, (cudaStream_t)stream);
   } else
     e = launch_down_stream(a, M, W_down, d, I, residual, out, status_word(workspace), *dev,
                            (cudaStream_t)stream);
@@ -265,8 +264,9 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
                             inited, done, status, *dev, s);
   } else if (use_tc(M, d, I, tile_T)) {
     const TcWorkspace tw = tc_workspace(workspace, L);
-    e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, tw, *dev, s);
-    if (e == cudaSuccess) e = launch_tc_down(a, M, W_down, d, I, residual, out, tw, *dev, s);
+    e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, out, residual, tw,
+                         *dev, s);
+    if (e == cudaSuccess) e = launch_tc_down(a, M, W_down, d, I, out, tw, *dev, s);
   } else {
     e = launch_gateup_stream(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, status, *dev, s);
     if (e == cudaSuccess)

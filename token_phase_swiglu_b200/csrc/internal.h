@@ -88,12 +88,20 @@ struct TcSizes {
 };
 TcSizes tc_sizes(int64_t M, int64_t d, int64_t I, int sm_count);
 bool tc_supported(int64_t M, int64_t d, int64_t I, int T);
+// The prologue of the gate-up GEMM also sets out_init (if not null) to the
+// residual (or zero) for a down GEMM that follows.
 cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float eps,
                              const void* P, int T, int64_t d, int64_t I, void* a,
-                             const TcWorkspace& ws, const DeviceInfo& dev, cudaStream_t stream);
+                             float* out_init, const void* residual, const TcWorkspace& ws,
+                             const DeviceInfo& dev, cudaStream_t stream);
+// out = residual or zero (for a down GEMM with no gate-up prologue before it).
+cudaError_t launch_out_init(float* out, const void* residual, int64_t M, int64_t d,
+                            const DeviceInfo& dev, cudaStream_t stream);
+// out += a W_down^T: split-K shares are added into out, which must already
+// hold the residual (or zero).
 cudaError_t launch_tc_down(const void* a, int64_t M, const void* W_down, int64_t d, int64_t I,
-                           const void* residual, float* out, const TcWorkspace& ws,
-                           const DeviceInfo& dev, cudaStream_t stream);
+                           float* out, const TcWorkspace& ws, const DeviceInfo& dev,
+                           cudaStream_t stream);
 
 // out[m, n] = sum_i W_down[n, i] a[m, i] (+ residual), same streaming scheme.
 cudaError_t launch_down_stream(const void* a, int64_t M, const void* W_down, int64_t d,

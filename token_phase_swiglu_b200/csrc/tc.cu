@@ -20,11 +20,13 @@
 //              accumulators double-buffered in TMEM, tcgen05.commit frees
 //              stages and publishes accumulators);
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//              lanes 32*(w%4)..+31), SwiGLU or residual add, stores.
-// Work is split "stream-K": the (tile, k-block) units are cut evenly over the
-// CTAs, so a tile may be shared by two or more CTAs; each writes its partial
-// accumulator to the workspace and the last one to arrive (tile counter) sums
-// them and runs the epilogue.  Nobody waits on another CTA.
+//              lanes 32*(w%4)..+31), SwiGLU and stores of a (gate-up), or
+//              red.add of the tile into out (down).
+// Work is split in data-parallel rounds of whole tiles and a "stream-K"
+// remainder (see the schedule below).  A gate-up tile shared by several CTAs
+// is finished by the last contributor from the others' partials (SwiGLU is
+// not linear); down-projection shares are simply added into out, which the
+// prologue set to the residual or zero.  Nobody waits on another CTA.
 // Every mbarrier wait is bounded; on expiry the CTA flags the status word,
 // waits for its own copies and MMAs, frees its TMEM and returns.
 #include "common.cuh"
@@ -232,8 +234,7 @@ struct TcParams {
   uint32_t tmem_cols;  // allocated TMEM columns (2 x C x N rounded up to a power of two)
   const float* rinv;   // [M] 1/RMS per token (SwiGLU)
   __nv_bfloat16* a_out;             // SwiGLU output a [M x I]
-  float* out;                       // down output [M x d]
-  const __nv_bfloat16* residual;    // [M x d] or null
+  float* out;                       // down output [M x d] (accumulated into)
   float* partials;     // [ctas][2][N][128] f32
   uint32_t* counters;  // [tiles] arrivals (zero between calls)
   uint32_t* status;
@@ -258,24 +259,11 @@ __device__ __forceinline__ void tc_flag(TcShared* sh, uint32_t* status) {
   atomicOr(status, kStatusTimeout);
 }
 
-// Epilogue of CW logical columns [col0, col0 + CW) of one finished tile
-// (warps 2-5; vals[j] = D[row, col0 + j], hi + lo already summed).
+// SwiGLU epilogue of CW logical columns [col0, col0 + CW) of one finished
+// gate-up tile (warps 2-5; vals[j] = D[row, col0 + j], hi + lo summed).
 template <int CW>
 __device__ __forceinline__ void epilogue_columns(const TcParams& p, int tt, int row,
                                                  const float (&vals)[CW], int col0) {
-  if (p.epi == kEpiDown) {
-    const int n = row;
-#pragma unroll
-    for (int j = 0; j < CW; ++j) {
-      const int m = tt * p.Mt + col0 + j;
-      if (m < p.M && n < p.d) {
-        float o = vals[j];
-        if (p.residual) o += __bfloat162float(p.residual[(int64_t)m * p.d + n]);
-        p.out[(int64_t)m * p.d + n] = o;
-      }
-    }
-    return;
-  }
   // SwiGLU: within a 2T-row interleave tile rows [0,T) are gate, [T,2T) up;
   // the partner row is lane ^ T (T in {8, 16}).  The gate lane finishes the
   // first half of the chunk's tokens, the up lane the second half.
@@ -352,6 +340,24 @@ __device__ void finish_tile(const TcParams& p, int t, uint32_t tb, bool whole, i
       }
     }
     epilogue_columns<CW>(p, tt, row, vals, c0);
+  }
+}
+
+// Down GEMM: add this CTA's accumulator of tile t (all C chains) into out.
+template <int CW>
+__device__ void add_tile_to_out(const TcParams& p, int t, uint32_t tb, int r_local) {
+  const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
+  const int n = rt * kBM + r_local;
+  for (int c0 = 0; c0 < p.N; c0 += CW) {
+    float v[CW];
+    tile_cols<CW>(p, tb, c0, v);
+    if (n < p.d) {
+#pragma unroll
+      for (int j = 0; j < CW; ++j) {
+        const int m = tt * p.Mt + c0 + j;
+        if (m < p.M) atomicAdd(p.out + (int64_t)m * p.d + n, v[j]);
+      }
+    }
   }
 }
 
@@ -516,7 +522,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
     const int r_local = 32 * q + lane;       // accumulator row = TMEM lane
     const int et = threadIdx.x - 64;         // 0..127
     const int ncol = p.epi == kEpiSwiGLU ? p.Mt : p.N;  // logical columns (hi + lo summed)
-    grid_dependency_wait();  // 1/RMS and the residual come from earlier kernels
+    grid_dependency_wait();  // 1/RMS and the initial out come from earlier kernels
     for (int s = 0; s < nseg; ++s) {
       int t, kb0, kb1;
       segment(p.sched, u0, u1, s, t, kb0, kb1);
@@ -527,6 +533,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
       if (epilogue_barrier_any(!got)) break;
       tc_fence_after();
       const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.C * p.N);
+      if (p.epi == kEpiDown) {
+        // Split-K by accumulation: out already holds the residual (or zero)
+        // and every contributor of a tile adds its share; no partials, no
+        // tile counters, nobody waits for the last contributor.
+        if (p.N % 32 == 0) add_tile_to_out<32>(p, t, tb, r_local);
+        else add_tile_to_out<16>(p, t, tb, r_local);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
+        continue;
+      }
       const bool whole = kb0 == 0 && kb1 == p.sched.KB;
       const int64_t tu = (int64_t)(t - p.sched.sk_tile0()) * p.sched.KB;  // stream-K tiles only
       const int c_first = whole ? 0 : p.sched.cta_of(tu);
@@ -592,9 +609,12 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
                                                  __nv_bfloat16* __restrict__ b_hl,
                                                  float* __restrict__ rinv,
                                                  uint32_t* __restrict__ counters,
-                                                 int ncounters) {
-  grid_dependency_wait();
+                                                 int ncounters, float* __restrict__ out,
+                                                 const __nv_bfloat16* __restrict__ residual) {
+  // The GEMM launched next may start (and prefetch its weights) right away;
+  // it waits for this grid's completion before it reads what this writes.
   grid_launch_dependents();
+  grid_dependency_wait();
   // The stream-K arrival counters start every call at zero, whatever a
   // previous call (an aborted one, or one of another shape) left there.  The
   // previous call's kernels are complete once the wait above returns.
@@ -628,6 +648,17 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
     reinterpret_cast<uint4*>(hi)[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     reinterpret_cast<uint4*>(lo)[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
+  // The down GEMM adds its split-K shares into out: start it at the residual
+  // (or zero), one token row per CTA.
+  if (out && m < M)
+    for (int v = threadIdx.x; v < d / 4; v += blockDim.x) {
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (residual) {
+        const uint2 r = __ldg(reinterpret_cast<const uint2*>(residual + (int64_t)m * d) + v);
+        o = make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+      }
+      reinterpret_cast<float4*>(out + (int64_t)m * d)[v] = o;
+    }
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -635,6 +666,24 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
     float t = 0.f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
     rinv[m] = 1.0f / sqrtf(t / (float)d + eps);
+  }
+}
+
+// out = residual (or zero), before a down GEMM that is not preceded by the
+// gate-up prologue (fmlp_down_proj).
+__global__ void __launch_bounds__(256) out_init(float* __restrict__ out,
+                                                const __nv_bfloat16* __restrict__ residual,
+                                                int64_t n4) {
+  grid_launch_dependents();
+  grid_dependency_wait();
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (residual) {
+      const uint2 r = __ldg(reinterpret_cast<const uint2*>(residual) + i);
+      o = make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+    }
+    reinterpret_cast<float4*>(out)[i] = o;
   }
 }
 
@@ -789,7 +838,8 @@ bool tc_supported(int64_t M, int64_t d, int64_t I, int T) {
 
 cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float eps,
                              const void* P, int T, int64_t d, int64_t I, void* a,
-                             const TcWorkspace& ws, const DeviceInfo& dev, cudaStream_t stream) {
+                             float* out_init, const void* residual, const TcWorkspace& ws,
+                             const DeviceInfo& dev, cudaStream_t stream) {
   const TcPlan pl = make_tc_plan(kEpiSwiGLU, M, d, dev);
   // prologue: hi/lo split of x * gamma into the token-tiled B operand, and 1/RMS
   {
@@ -805,7 +855,7 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
     cudaError_t e = cudaLaunchKernelEx(&cfg, act_split, (const __nv_bfloat16*)x,
                                        (const __nv_bfloat16*)gamma, eps, (int)M, (int)d, pl.Mt,
                                        (__nv_bfloat16*)ws.b_hl, ws.rinv, ws.counters,
-                                       ws.ncounters);
+                                       ws.ncounters, out_init, (const __nv_bfloat16*)residual);
     if (e != cudaSuccess) return e;
     note_launches(1);
   }
@@ -827,9 +877,27 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
   return launch_tc(p, pl, dev, stream);
 }
 
+cudaError_t launch_out_init(float* out, const void* residual, int64_t M, int64_t d,
+                            const DeviceInfo& dev, cudaStream_t stream) {
+  const int64_t n4 = M * d / 4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256,
+                                                                       4 * dev.sm_count)));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, out_init, out, (const __nv_bfloat16*)residual, n4);
+  if (e == cudaSuccess) note_launches(1);
+  return e;
+}
+
 cudaError_t launch_tc_down(const void* a, int64_t M, const void* W_down, int64_t d, int64_t I,
-                           const void* residual, float* out, const TcWorkspace& ws,
-                           const DeviceInfo& dev, cudaStream_t stream) {
+                           float* out, const TcWorkspace& ws, const DeviceInfo& dev,
+                           cudaStream_t stream) {
   const TcPlan pl = make_tc_plan(kEpiDown, M, I, dev);
   TcParams p;
   memset(&p, 0, sizeof(p));
@@ -843,7 +911,6 @@ cudaError_t launch_tc_down(const void* a, int64_t M, const void* W_down, int64_t
   p.I = (int)I;
   p.d = (int)d;
   p.out = out;
-  p.residual = (const __nv_bfloat16*)residual;
   return launch_tc(p, pl, dev, stream);
 }
 
