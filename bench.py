@@ -67,10 +67,18 @@ def measured_peaks() -> dict:
         return {}
 
 
-def kernel_source_hash() -> str:
+# the source files each kernel is built from (its traffic record goes stale
+# when any of them changes)
+KERNEL_SOURCES = {
+    "fused_decode": ["stream.cu", "common.cuh", "internal.h"],
+    "tc_gemm": ["tc.cu", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "token_phase_swiglu_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -84,7 +92,7 @@ def recorded_traffic(kernel: str, workload: str):
             rec = json.load(f).get(kernel, {}).get(workload)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or kernel not in KERNEL_SOURCES or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -457,7 +465,7 @@ def run_ours(args) -> None:
         else:
             bound, kpeak, kpeak_src, kunit, kwork = "hbm", peak, peak_src, "GB/s", kbytes
     k_achieved = kwork / (kms / 1e3) / (1e12 if kunit == "TFLOP/s" else 1e9)
-    traffic = recorded_traffic(kname, w.name)
+    traffic = recorded_traffic("fused_decode" if fused else "tc_gemm", w.name)
 
     if rank == 0:
         cpu = None
