@@ -106,7 +106,16 @@ FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
  * Precision: x*gamma is formed exactly in f32 and the contraction keeps it at
  * f32 precision (CUDA-core path) or as an exact hi+lo bf16 pair (tensor-core
  * path); accumulation is f32; a is rounded once to bf16 (round to nearest
- * even); out is f32.
+ * even); out is f32.  out is written by several thread blocks adding into it
+ * (f32 atomics), so the summation order, and the last bits of out, may differ
+ * from run to run.  out must not overlap any input.
+ *
+ * Ordering: the kernels use programmatic dependent launch.  A kernel of this
+ * library may start streaming packed_Wgu, W_down and gamma while the
+ * previous kernel on the stream is still running, if that kernel is one of
+ * this library's (fmlp_pack excepted), which never write those buffers.
+ * Everything else (x, residual, out, workspace) is touched only after the
+ * previous work on the stream has completed.
  */
 FMLP_API fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
                          const void* packed_Wgu, int tile_T, const void* W_down,
