@@ -274,6 +274,35 @@ def test_side_stream_and_workspace_reuse(fm):
     assert fm.fmlp_device_status(ws) == fm.FMLP_OK
 
 
+def test_concurrent_streams_do_not_wait_on_each_other(fm):
+    """Two single-launch decode calls on two streams at once, each with its
+    own workspace and weights large enough that every thread block needs a
+    whole SM: the kernel never waits for a thread block that has not been
+    scheduled, so both finish correctly (no bounded wait expires) however
+    the hardware interleaves their blocks."""
+    dev = torch.device("cuda:0")
+    d, I, T = 3072, 8192, 16
+    runs = []
+    for k in range(2):
+        p = wl.make_problem(1, d, I, seed=90 + k, residual=k == 1)
+        g = {n: v.to(dev) for n, v in p.items()}
+        packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+        fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+        ws = torch.zeros(fm.fmlp_workspace_bytes(1, d, I), dtype=torch.uint8, device=dev)
+        out = torch.empty(1, d, dtype=torch.float32, device=dev)
+        runs.append((p, g, packed, ws, out, torch.cuda.Stream()))
+    torch.cuda.synchronize()
+    for _ in range(50):
+        for k, (p, g, packed, ws, out, st) in enumerate(runs):
+            with torch.cuda.stream(st):
+                fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, T, g["W_down"], out, ws,
+                                residual=g["residual"] if k == 1 else None, stream=st)
+    torch.cuda.synchronize()
+    for k, (p, g, packed, ws, out, st) in enumerate(runs):
+        assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+        assert_parity(out.cpu().double().numpy(), oracle_out(p, residual=k == 1))
+
+
 def test_workspace_reuse_across_paths(fm):
     """One workspace, zeroed once, serves calls of any M and I at a fixed d:
     the fused decode kernel, the tensor-core GEMMs and the streaming kernels

@@ -106,6 +106,7 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
   L.status = off;
   L.inited = off + 64;
   L.done = off + 128;
+  L.ticket = off + 192;
   off += 256;
   L.zero_end = off;
   L.a = off;
@@ -258,10 +259,11 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   if (fused_decode_supported(M, d, I, *dev)) {
+    uint32_t* ticket = (uint32_t*)((char*)workspace + L.ticket);
     uint32_t* inited = (uint32_t*)((char*)workspace + L.inited);
     uint32_t* done = (uint32_t*)((char*)workspace + L.done);
     e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out,
-                            inited, done, status, *dev, s);
+                            ticket, inited, done, status, *dev, s);
   } else if (use_tc(M, d, I, tile_T)) {
     const TcWorkspace tw = tc_workspace(workspace, L);
     e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, out, residual, tw,

@@ -20,15 +20,16 @@ struct DeviceInfo {
 cudaError_t current_device_info(const DeviceInfo** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
-// The first 256 bytes are control words: the device status word at 0, the
-// fused kernel's out-initialised counter at 64 and finished-CTA counter at
-// 128.  They must read zero when a call starts and every call (a timed-out
-// one too) leaves them at zero, so one workspace serves calls of any M, d
-// and I that fit in it.
+// The first 256 bytes are control words: the device status word at 0, and
+// the fused kernel's counters: out shares set at 64, finished CTAs at 128,
+// arrival tickets at 192.  They must read zero when a call starts and every
+// call (a timed-out one too) leaves them at zero, so one workspace serves
+// calls of any M, d and I that fit in it.
 struct WorkspaceLayout {
   size_t status = 0;     // uint32 device status word
-  size_t inited = 64;    // uint32 CTAs whose share of out is set (fused kernel)
+  size_t inited = 64;    // uint32 out shares set (fused kernel)
   size_t done = 128;     // uint32 finished-CTA counter (fused kernel)
+  size_t ticket = 192;   // uint32 CTA arrival tickets (fused kernel)
   size_t zero_end = 256;
   size_t a = 0;          // bf16 [M x I] intermediate
   size_t b_hl = 0, rinv = 0, partials = 0, counters = 0;  // tensor-core path
@@ -64,14 +65,15 @@ cudaError_t launch_gateup_stream(const void* x, int64_t M, const void* gamma, fl
 
 // Both steps in one launch, split over the intermediate dimension (M <= 4,
 // fused_decode_supported).  CTAs add their partial down projections into
-// out; inited / done: the workspace's counters of CTAs that have set their
-// share of out and of CTAs finished, zero on entry and on exit.
+// out once the first CTAs to arrive have set it; ticket / inited / done: the
+// workspace's counters of arrivals, of out shares set and of CTAs finished,
+// zero on entry and on exit.
 bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev);
 cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                                const void* residual, float* out, uint32_t* inited,
-                                uint32_t* done, uint32_t* status, const DeviceInfo& dev,
-                                cudaStream_t stream);
+                                const void* residual, float* out, uint32_t* ticket,
+                                uint32_t* inited, uint32_t* done, uint32_t* status,
+                                const DeviceInfo& dev, cudaStream_t stream);
 
 // Tensor-core path (tcgen05, csrc/tc.cu) for M above the decode range.
 constexpr int kTcMaxCtas = 160;  // workspace sizing bound on the grid (>= SMs of a B200)

@@ -614,8 +614,10 @@ struct FusedParams {
   const __nv_bfloat16* gamma;
   const __nv_bfloat16* residual;
   float* out;          // [M x d] f32: set to the residual (or 0), then CTAs add into it
-  uint32_t* inited;    // CTAs whose share of out is set (zero between calls)
+  uint32_t* ticket;    // arrival order of the CTAs (zero between calls)
+  uint32_t* inited;    // initialising CTAs whose share of out is set (zero between calls)
   uint32_t* done;      // CTAs finished (zero between calls)
+  int n_init;          // CTAs that initialise out: the first n_init to arrive
   Control ctl;
   GateUpGeom gu;
   float eps;
@@ -716,12 +718,20 @@ __device__ bool wait_counter(const uint32_t* ctr, uint32_t target, uint64_t limi
   }
 }
 
-// Warp 0, lanes 1-31: this CTA's share of out (float4 granules) set to the
-// residual or to zero, then counted in `inited`.
+// Warp 0, lanes 1-31.  The first n_init CTAs to arrive (an atomic ticket,
+// taken once the previous kernel on the stream is done) set one share each
+// of out (float4 granules) to the residual or zero and count it in inited.
+// The consumers of every CTA wait for that count before adding into out; as
+// the initialising CTAs are by construction already running, nobody waits
+// on a CTA that has not been scheduled, so no co-residency is assumed.
 __device__ void init_out_share(const FusedParams& p, int mt, int lane) {
-  grid_dependency_wait();  // out and the residual belong to the stream's order
+  grid_dependency_wait();  // out, the residual and the counters belong to this call now
+  uint32_t t = 0;
+  if (lane == 1) t = atomicAdd(p.ticket, 1u);
+  t = __shfl_sync(0xfffffffeu, t, 1);
+  if (t >= (uint32_t)p.n_init) return;
   const int64_t n4 = (int64_t)mt * p.d / 4;
-  const int64_t q0 = n4 * blockIdx.x / gridDim.x, q1 = n4 * (blockIdx.x + 1) / gridDim.x;
+  const int64_t q0 = n4 * t / p.n_init, q1 = n4 * (t + 1) / p.n_init;
   for (int64_t i = q0 + lane - 1; i < q1; i += 31) {
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (p.residual) {
@@ -782,13 +792,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
     stage_x_gamma<MT>(p.x, nullptr, p.eps, p.d, 0, mt, s, red, rinv);
     const bool ok = consume_gateup<MT>(cs, p.gu, g0, ng, s, rinv, nullptr, 0, mt, xch, slice,
                                        i0, p.swbox);
-    // Every CTA's share of out must be set before anyone adds into it.  The
-    // shares are written at the start, so by the end of the gate-up phase
-    // this normally returns at once (the ring keeps filling meanwhile).  The
-    // decision is published before the barrier so all consumer warps take it.
+    // All of out must be set before anyone adds into it.  The shares are
+    // written at the start by CTAs already running, so by the end of the
+    // gate-up phase this normally returns at once (the ring keeps filling
+    // meanwhile).  The decision is published before the barrier so all
+    // consumer warps take it.
     if (ct == 0) {
       bool g = ok;
-      if (g && !wait_counter(p.inited, gridDim.x, p.ctl.wait_ns, &st.abort)) {
+      if (g && !wait_counter(p.inited, (uint32_t)p.n_init, p.ctl.wait_ns, &st.abort)) {
         flag_timeout(&st, p.ctl.status);
         g = false;
       }
@@ -801,10 +812,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
   __syncthreads();
   if (threadIdx.x == 0) {
     if (st.abort) drain_ring(ring, st.issued);
-    // Every CTA has counted itself in `inited` and is past its wait on it:
-    // the last one to get here leaves both counters at zero for the next call
-    // (also after a timeout).
+    // Every CTA has taken its ticket, finished any share of out it owned and
+    // is past its wait on `inited`: the last one to get here leaves the
+    // counters at zero for the next call (also after a timeout).
     if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+      atomicExch(p.ticket, 0u);
       atomicExch(p.inited, 0u);
       atomicExch(p.done, 0u);
     }
@@ -1037,9 +1049,9 @@ bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& d
 
 cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                                const void* residual, float* out, uint32_t* inited,
-                                uint32_t* done, uint32_t* status, const DeviceInfo& dev,
-                                cudaStream_t stream) {
+                                const void* residual, float* out, uint32_t* ticket,
+                                uint32_t* inited, uint32_t* done, uint32_t* status,
+                                const DeviceInfo& dev, cudaStream_t stream) {
   const FusedPlan f = make_fused_plan(M, d, I, dev);
   if (f.mt == 0) return cudaErrorInvalidConfiguration;
   FusedParams p;
@@ -1052,8 +1064,10 @@ cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, flo
   p.gamma = (const __nv_bfloat16*)gamma;
   p.residual = (const __nv_bfloat16*)residual;
   p.out = out;
+  p.ticket = ticket;
   p.inited = inited;
   p.done = done;
+  p.n_init = std::min(f.grid, 4);
   p.ctl.status = status;
   p.ctl.wait_ns = wait_timeout_ns();
   p.ctl.drop_last = fault_injection();
