@@ -717,33 +717,30 @@ void tc_shape(int epi, int64_t M, int& Mt, int& N, int& C) {
   C = 4 * N <= 256 ? 4 : (2 * N <= 256 ? 2 : 1);
 }
 
-#ifndef FMLP_TC_MAX_KS
-#define FMLP_TC_MAX_KS 4
-#endif
-#ifndef FMLP_TC_MIN_STAGES
-#define FMLP_TC_MIN_STAGES 2
-#endif
+constexpr int kTcMaxKs = 4;
 
 // Stages of KS k-blocks.  On B200 one SM issues TMA copies at a few million
 // per second whatever their size (measured: ~2 M stages/s of two copies),
-// so a stage moves KS k-blocks of A and of B in one copy each, with KS as
-// large as still leaves FMLP_TC_MIN_STAGES stages: on the 8B-shaped decode
-// layers fewer, larger copies beat a deeper ring of small ones (M = 8:
-// 3.2 -> 5.0 TB/s).
+// so a stage moves KS k-blocks of A and of B in one copy each.  KS is the
+// largest that still leaves a ring of 3 stages for narrow B operands (decode
+// batches: 8B M = 8 went from 3.2 to 5.4 TB/s, M = 32 gains 4% from 3 stages
+// of 3 k-blocks over 2 of 4) and of 2 stages for wide ones (verify, prefill:
+// deeper rings of single k-blocks were 6-13% slower there).
 TcPlan make_tc_plan(int epi, int64_t M, int64_t K, const DeviceInfo& dev) {
   TcPlan pl;
   tc_shape(epi, M, pl.Mt, pl.N, pl.C);
   pl.ntok = (int)((M + pl.Mt - 1) / pl.Mt);
   const size_t budget = (size_t)dev.max_smem_optin - 2048 - 1024;  // static + alignment slack
   const int kb_total = (int)(K / kBK);
-  for (int ks = FMLP_TC_MAX_KS; ks >= 1; ks /= 2) {
+  const int min_stages = pl.N < 128 ? 3 : 2;
+  for (int ks = kTcMaxKs; ks >= 1; --ks) {
     if (ks > 1 && ks > kb_total) continue;
     pl.KS = ks;
     pl.a_bytes = ks * kATileBytes;
     pl.b_bytes = ks * pl.N * kBK * 2;
     pl.stage_bytes = (pl.a_bytes + pl.b_bytes + 1023) / 1024 * 1024;
     pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
-    if (pl.stages >= FMLP_TC_MIN_STAGES) break;
+    if (pl.stages >= min_stages) break;
   }
   pl.smem = (size_t)pl.stages * pl.stage_bytes + 1024;
   pl.tmem_cols = pow2_at_least((uint32_t)(2 * pl.C * pl.N));
