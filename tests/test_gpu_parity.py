@@ -434,6 +434,7 @@ TC_CASES = [
     (24, 512, 1024, 16, True),    # 4 row sub-tiles, 16-column epilogue chunks
     (72, 256, 512, 8, False),     # one row sub-tile, 8-column chunks, 16-column partial tail
     (40, 640, 1280, 16, True),    # 2 row sub-tiles (gate-up), 8-column chunks
+    (256, 512, 9600, 16, True),   # 300 gate-up tiles: a data-parallel wave, then stream-K
 ]
 
 
@@ -444,6 +445,28 @@ def test_tensor_core_path(fm, M, d, I, T, residual):
     got = run_forward(fm, p, T=T, residual=residual)
     ref = oracle_out(p, residual=residual)
     assert_parity(got, ref, oracle_out(p, residual=residual, intermediate="bf16"))
+
+
+@pytest.mark.parametrize("M,d,I", [(24, 512, 1024), (130, 384, 640)])
+def test_tensor_core_down_proj_alone(fm, M, d, I):
+    """fmlp_down_proj on the tensor path sets out to the residual (or zero)
+    itself and then adds the split-K shares: compare with a binary64 product,
+    with and without residual, twice into the same out buffer."""
+    dev = torch.device("cuda:0")
+    a = wl.normal_bf16(6, 0, (M, I))
+    Wd = wl.normal_bf16(6, 4, (d, I), std=0.02)
+    res = wl.normal_bf16(6, 5, (M, d))
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    out = torch.full((M, d), float("nan"), dtype=torch.float32, device=dev)
+    for with_res in (True, False, True):
+        fm.fmlp_down_proj(a.to(dev), Wd.to(dev), out, ws, residual=res.to(dev) if with_res else None)
+        torch.cuda.synchronize()
+        ref = oracle.decode_bf16(bits(a)) @ oracle.decode_bf16(bits(Wd)).T
+        if with_res:
+            ref = ref + oracle.decode_bf16(bits(res))
+        norm, _ = errors(out.cpu().double().numpy(), ref)
+        assert norm <= 1e-5
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
 
 
 def test_tensor_core_stage_calls(fm):
