@@ -298,9 +298,11 @@ def run_ours(args) -> None:
     M, d, I, L = w.M, w.d, w.I, (args.layers or w.layers)
     seed0 = 1000 * rank
 
-    # resident weights: packed gate/up and W_down per layer (+ gamma per layer)
+    # resident weights: packed gate/up and W_down per layer (+ gamma per layer);
+    # the layers' outputs are slices of one buffer, returned with one copy
     act = wl.make_activations(M, d, seed=seed0)
     x = act["x"].to(dev)
+    outs = torch.empty(L, M, d, dtype=torch.float32, device=dev)
     layers = []
     for l in range(L):
         wts = wl.make_weights(d, I, w.sigma, seed=seed0 + l)
@@ -311,7 +313,7 @@ def run_ours(args) -> None:
         torch.cuda.synchronize()
         del wg, wu
         layers.append({"packed": packed, "W_down": wts["W_down"].to(dev), "gamma": gamma,
-                       "out": torch.empty(M, d, dtype=torch.float32, device=dev)})
+                       "out": outs[l]})
     ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
     a_buf = torch.empty(M, I, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -422,8 +424,7 @@ def run_ours(args) -> None:
         for li, ly in enumerate(layers):
             fm.fmlp_forward(x_dev, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], ly["out"],
                             ws, stream=stream)
-        for li, ly in enumerate(layers):
-            outs_host[li].copy_(ly["out"], non_blocking=True)
+        outs_host.copy_(outs, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
