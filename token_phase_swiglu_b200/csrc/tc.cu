@@ -47,6 +47,9 @@ constexpr int kBK = 64;         // k-block: one 128-byte swizzle atom of bf16
 constexpr int kATileBytes = kBM * kBK * 2;
 constexpr int kMaxStages = 12;
 constexpr uint64_t kDrainNs = 1000000000ull;
+// Pair kernel teardown: a stage one CTA issued but the leader never armed
+// never completes; its copies land within microseconds, so a short limit.
+constexpr uint64_t kPairDrainNs = 2000000ull;
 
 enum Epi { kEpiSwiGLU = 0, kEpiDown = 1 };
 
@@ -181,12 +184,6 @@ struct Sched {
     const int64_t U = units(), per = U / ctas, rem = U % ctas;
     const int64_t big = rem * (per + 1);
     return u < big ? (int)(u / (per + 1)) : (int)(rem + (u - big) / per);
-  }
-  // first tile of CTA c's stream-K range
-  __device__ __forceinline__ int sk_first_tile(int c) const {
-    int64_t u0, u1;
-    range(c, u0, u1);
-    return sk_tile0() + (int)(u0 / KB);
   }
 };
 
@@ -599,6 +596,405 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
 }
 
 // ---------------------------------------------------------------------------
+// Two-SM tiles (cta_group::2) for wide operands (N >= 128: verify, prefill).
+//
+// A cluster of two CTAs computes a 256-row tile: CTA r holds weight rows
+// [128 r, 128 r + 128) of the tile and rows [N/2 r, N/2 r + N/2) of the B
+// operand in its shared memory, and its TMEM holds the 128 x N accumulator
+// of its rows.  Per k-block each CTA loads 16 KB of weights and N/2 x 128 B
+// of activations instead of N x 128 B: half the activation traffic per
+// weight byte of the one-SM kernel.  Both CTAs load their own halves and
+// signal the leader's (rank 0) "full" barrier, which the leader's producer
+// arms with both CTAs' bytes; the leader's MMA warp issues every MMA
+// (tcgen05.mma.cta_group::2, M = 256) and its commits arrive on both CTAs'
+// "empty" and "accumulator full" barriers; both epilogues release the
+// accumulator on the leader's barrier.  Stream-K partials and tile counters
+// are kept per (tile, rank).
+// Teardown: both CTAs stop, meet at a cluster barrier, the leader waits for
+// every stage either CTA issued (bounded) and for its MMAs, and a second
+// cluster barrier precedes TMEM release and exit, so no copy, MMA or
+// barrier arrive of one CTA can target a CTA that has left.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// 3-D TMA copy into this CTA's shared memory whose completion is counted on
+// the pair leader's barrier (a shared::cluster address).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const void* tmap, int x, int y, int z,
+                                                 uint32_t leader_bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;"
+      ::"r"(smem_u32(dst)), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(leader_bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// arrive (when the leader's MMAs issued so far complete) on the barrier at
+// the same offset in the CTAs of `mask`
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)), "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Segment s of stream-K/data-parallel work unit `me` (a CTA, or a CTA pair).
+__device__ __forceinline__ bool segment_of(const Sched& S, int me, int64_t u0, int64_t u1, int s,
+                                           int& t, int& kb0, int& kb1) {
+  if (s < S.dp) {
+    t = s * S.ctas + me;
+    kb0 = 0;
+    kb1 = S.KB;
+    return true;
+  }
+  s -= S.dp;
+  if (u0 >= u1) return false;
+  const int tl = (int)(u0 / S.KB) + s;
+  const int64_t tb = (int64_t)tl * S.KB;
+  if (tb >= u1) return false;
+  t = S.sk_tile0() + tl;
+  kb0 = (int)(max(u0, tb) - tb);
+  kb1 = (int)(min(u1, tb + S.KB) - tb);
+  return true;
+}
+
+// Finish this CTA's 128 rows of a gate-up tile in the pair kernel: its
+// accumulator plus the other pairs' partials of the same rank.
+template <int CW>
+__device__ void finish_tile_pair(const TcParams& p, int t, int rank, uint32_t tb, bool whole,
+                                 int c_first, int c_last, int me, int r_local) {
+  const int ncol = p.Mt;
+  const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
+  const int row = rt * 2 * kBM + rank * kBM + r_local;
+  for (int c0 = 0; c0 < ncol; c0 += CW) {
+    float vals[CW];
+    tile_cols<CW>(p, tb, c0, vals);
+    float lo[CW];
+    tile_cols<CW>(p, tb, p.Mt + c0, lo);  // lo half of x*gamma
+#pragma unroll
+    for (int j = 0; j < CW; ++j) vals[j] += lo[j];
+    if (!whole) {
+      for (int cc = c_first; cc <= c_last; ++cc) {
+        if (cc == me) continue;
+        int64_t cu0, cu1;
+        p.sched.range(cc, cu0, cu1);
+        const int slot = (t == p.sched.sk_tile0() + (int)(cu0 / p.sched.KB)) ? 0 : 1;
+        const float* part =
+            p.partials + ((size_t)(cc * 2 + rank) * 2 + slot) * (size_t)p.N * kBM;
+#pragma unroll
+        for (int j = 0; j < CW; ++j)
+          vals[j] += __ldcg(part + (size_t)(c0 + j) * kBM + r_local) +
+                     __ldcg(part + (size_t)(p.Mt + c0 + j) * kBM + r_local);
+      }
+    }
+    epilogue_columns<CW>(p, tt, row, vals, c0);
+  }
+}
+
+template <int CW>
+__device__ void add_tile_to_out_pair(const TcParams& p, int t, int rank, uint32_t tb,
+                                     int r_local) {
+  const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
+  const int n = rt * 2 * kBM + rank * kBM + r_local;
+  for (int c0 = 0; c0 < p.N; c0 += CW) {
+    float v[CW];
+    tile_cols<CW>(p, tb, c0, v);
+    if (n < p.d) {
+#pragma unroll
+      for (int j = 0; j < CW; ++j) {
+        const int m = tt * p.Mt + c0 + j;
+        if (m < p.M) atomicAdd(p.out + (int64_t)m * p.d + n, v[j]);
+      }
+    }
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+    tc_gemm_pair(const __grid_constant__ TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ TcShared sh;
+  uint8_t* stage0 = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = (int)cluster_ctarank();
+  const bool leader = rank == 0;
+  const int me = (int)blockIdx.x / 2;  // the pair's work index
+  const int N = p.N, half_n = p.N / 2;
+  int64_t u0, u1;
+  p.sched.range(me, u0, u1);
+  int nseg = 0, nk = 0;
+  {
+    int t, a, b;
+    while (segment_of(p.sched, me, u0, u1, nseg, t, a, b)) {
+      nk += b - a;
+      ++nseg;
+    }
+  }
+
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < p.stages; ++j) {
+      mbar_init(&sh.full[j], 1);   // the leader's producer arms it (both CTAs' bytes)
+      mbar_init(&sh.empty[j], 1);  // one multicast commit per stage
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&sh.acc_full[j], 1);
+      mbar_init(&sh.acc_empty[j], 8);  // four epilogue warps of each CTA (leader's is used)
+    }
+    mbar_init(&sh.mma_done, 1);
+    sh.abort = 0;
+    sh.k_issued = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc_pair(&sh.tmem_base, p.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any copy or arrive targets them
+  tc_fence_after();
+  grid_launch_dependents();
+  const uint32_t tmem = sh.tmem_base;
+  volatile int* abort = &sh.abort;
+  const uint32_t leader_full = mapa_shared(&sh.full[0], 0);
+  const uint32_t leader_acc_empty = mapa_shared(&sh.acc_empty[0], 0);
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      const uint64_t pol_a = evict_first_policy();
+      uint64_t pol_b;
+      asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_b));
+      const int a_row0 = rank * kBM, b_row0 = rank * half_n;
+      int early_kb[kMaxStages], early_tt[kMaxStages];
+      const int n_early = min(nk, p.stages) - (p.drop_last && nk <= p.stages ? 1 : 0);
+      int k = 0;
+      bool ok = true;
+      for (int s = 0; s < nseg && ok && !*abort; ++s) {
+        int t, kb0, kb1;
+        segment_of(p.sched, me, u0, u1, s, t, kb0, kb1);
+        const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
+        for (int kb = kb0; kb < kb1; ++kb, ++k) {
+          if (p.drop_last && k == nk - 1) {
+            ok = false;
+            break;
+          }
+          const int slot = k % p.stages;
+          uint8_t* a_dst = stage0 + (size_t)slot * p.stage_bytes;
+          uint8_t* b_dst = a_dst + p.a_bytes;
+          if (k >= p.stages) {
+            if (k == p.stages) {
+              grid_dependency_wait();  // activations of the early stages
+              for (int e = 0; e < n_early; ++e)
+                tma_load_3d_pair(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map, 0,
+                                 early_tt[e] * N + b_row0, early_kb[e] * p.KS,
+                                 leader_full + 8u * e, pol_b);
+            }
+            if (!mbar_wait_bounded(&sh.empty[slot], (uint32_t)(((k / p.stages) - 1) & 1),
+                                   p.wait_ns, abort)) {
+              tc_flag(&sh, p.status);
+              ok = false;
+              break;
+            }
+          }
+          if (leader)
+            mbar_arrive_expect_tx(&sh.full[slot], (uint32_t)(2 * (p.a_bytes + p.b_bytes)));
+          tma_load_3d_pair(a_dst, &p.a_map, 0, rt * 2 * kBM + a_row0, kb * p.KS,
+                           leader_full + 8u * slot, pol_a);
+          if (k < p.stages) {
+            early_kb[k] = kb;
+            early_tt[k] = tt;
+          } else {
+            tma_load_3d_pair(b_dst, &p.b_map, 0, tt * N + b_row0, kb * p.KS,
+                             leader_full + 8u * slot, pol_b);
+          }
+          sh.k_issued = k + 1;
+        }
+      }
+      if (k <= p.stages && k > 0) {
+        grid_dependency_wait();
+        for (int e = 0; e < k; ++e)
+          tma_load_3d_pair(stage0 + (size_t)e * p.stage_bytes + p.a_bytes, &p.b_map, 0,
+                           early_tt[e] * N + b_row0, early_kb[e] * p.KS, leader_full + 8u * e,
+                           pol_b);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader only) ----------------
+    if (leader && lane == 0) {
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+                             ((uint32_t)((2 * kBM) >> 4) << 24);
+      int k = 0;
+      bool ok = true;
+      for (int s = 0; s < nseg && ok; ++s) {
+        int t, kb0, kb1;
+        segment_of(p.sched, me, u0, u1, s, t, kb0, kb1);
+        const int buf = s & 1;
+        if (!mbar_wait_bounded(&sh.acc_empty[buf], (uint32_t)(((s >> 1) & 1) ^ 1), p.wait_ns,
+                               abort)) {
+          tc_flag(&sh, p.status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * p.C * N);
+        for (int kb = kb0; kb < kb1; ++kb, ++k) {
+          const int slot = k % p.stages;
+          if (!mbar_wait_bounded(&sh.full[slot], (uint32_t)((k / p.stages) & 1), p.wait_ns,
+                                 abort)) {
+            tc_flag(&sh, p.status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stage0 + (size_t)slot * p.stage_bytes);
+          const uint32_t b_addr = a_addr + p.a_bytes;
+          const uint32_t b_kblock = (uint32_t)(half_n * kBK * 2);
+          const int nkb = min(p.KS, p.KBtot - kb * p.KS);
+          for (int kbi = 0; kbi < nkb; ++kbi) {
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const int c = kk % p.C;
+              const bool first = kb == kb0 && kbi == 0 && kk < p.C;
+              mma_bf16_pair(d_tmem + (uint32_t)(c * N),
+                            sw128_desc(a_addr + (uint32_t)(kbi * kATileBytes) + kk * 32),
+                            sw128_desc(b_addr + (uint32_t)kbi * b_kblock + kk * 32), idesc,
+                            first ? 0u : 1u);
+            }
+          }
+          mma_commit_pair(&sh.empty[slot], (uint16_t)3);  // both CTAs' slot reusable
+        }
+        if (ok) mma_commit_pair(&sh.acc_full[buf], (uint16_t)3);
+      }
+      mma_commit_pair(&sh.mma_done, (uint16_t)1);
+      mbar_wait_bounded(&sh.mma_done, 0, kDrainNs, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2-5, both CTAs) ----------------
+    const int q = warp & 3;
+    const int r_local = 32 * q + lane;
+    const int et = threadIdx.x - 64;
+    const int ncol = p.epi == kEpiSwiGLU ? p.Mt : N;
+    grid_dependency_wait();  // 1/RMS and the initial out come from earlier kernels
+    for (int s = 0; s < nseg; ++s) {
+      int t, kb0, kb1;
+      segment_of(p.sched, me, u0, u1, s, t, kb0, kb1);
+      const int buf = s & 1;
+      const bool got =
+          mbar_wait_bounded(&sh.acc_full[buf], (uint32_t)((s >> 1) & 1), p.wait_ns, abort);
+      if (!got && lane == 0) tc_flag(&sh, p.status);
+      if (epilogue_barrier_any(!got)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.C * N);
+      if (p.epi == kEpiDown) {
+        if (N % 32 == 0) add_tile_to_out_pair<32>(p, t, rank, tb, r_local);
+        else add_tile_to_out_pair<16>(p, t, rank, tb, r_local);
+      } else {
+        const bool whole = kb0 == 0 && kb1 == p.sched.KB;
+        const int64_t tu = (int64_t)(t - p.sched.sk_tile0()) * p.sched.KB;
+        const int c_first = whole ? 0 : p.sched.cta_of(tu);
+        const int c_last = whole ? 0 : p.sched.cta_of(tu + p.sched.KB - 1);
+        bool finalize = whole;
+        if (!whole) {
+          const int slot = (t == p.sched.sk_tile0() + (int)(u0 / p.sched.KB)) ? 0 : 1;
+          float* part = p.partials + ((size_t)blockIdx.x * 2 + slot) * (size_t)N * kBM;
+          int c = 0;
+          for (; c + 32 <= N; c += 32) {
+            float v[32];
+            tile_cols<32>(p, tb, c, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) __stcg(part + (size_t)(c + j) * kBM + r_local, v[j]);
+          }
+          if (c < N) {  // N is a multiple of 16
+            float v[16];
+            tile_cols<16>(p, tb, c, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) __stcg(part + (size_t)(c + j) * kBM + r_local, v[j]);
+          }
+          __threadfence();
+          named_barrier_sync(1, 128);
+          if (et == 0)
+            sh.last = atomicAdd(p.counters + 2 * t + rank, 1u) == (uint32_t)(c_last - c_first);
+          named_barrier_sync(1, 128);
+          finalize = sh.last;
+          if (finalize) __threadfence();
+        }
+        if (finalize) {
+          if (ncol % 32 == 0)
+            finish_tile_pair<32>(p, t, rank, tb, whole, c_first, c_last, me, r_local);
+          else if (ncol % 16 == 0)
+            finish_tile_pair<16>(p, t, rank, tb, whole, c_first, c_last, me, r_local);
+          else
+            finish_tile_pair<8>(p, t, rank, tb, whole, c_first, c_last, me, r_local);
+          if (!whole && et == 0) atomicExch(p.counters + 2 * t + rank, 0u);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&sh.acc_empty[buf]);
+        else mbar_arrive_cluster(leader_acc_empty + 8u * buf);
+      }
+    }
+  }
+  __syncthreads();
+  cluster_sync();  // neither CTA issues anything any more
+  if (leader && threadIdx.x == 0) {
+    // Every stage either CTA issued counts its copies on this CTA's barriers:
+    // wait for them (bounded) before either CTA may leave.
+    const int mine = sh.k_issued;
+    const int peer = (int)ld_shared_cluster_u32(mapa_shared(&sh.k_issued, 1));
+    const int n = max(mine, peer);
+    for (int k = max(0, n - p.stages); k < n; ++k)
+      mbar_wait_bounded(&sh.full[k % p.stages], (uint32_t)((k / p.stages) & 1), kPairDrainNs,
+                        nullptr);
+  }
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, p.tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Prologue: B operand of the gate-up GEMM and 1/RMS per token.
 // One CTA per token slot of the padded token tiles: rows [2Mt*j + i] = hi and
 // [2Mt*j + Mt + i] = lo of token m = Mt*j + i (zeros for padding slots).
@@ -693,6 +1089,7 @@ __global__ void __launch_bounds__(256) out_init(float* __restrict__ out,
 struct TcPlan {
   int N = 0, Mt = 0, ntok = 0, C = 0, KS = 1, stages = 0, stage_bytes = 0, a_bytes = 0,
       b_bytes = 0;
+  bool pair = false;   // two-SM tiles (tc_gemm_pair)
   uint32_t tmem_cols = 0;
   size_t smem = 0;
 };
@@ -732,12 +1129,17 @@ TcPlan make_tc_plan(int epi, int64_t M, int64_t K, const DeviceInfo& dev) {
   pl.ntok = (int)((M + pl.Mt - 1) / pl.Mt);
   const size_t budget = (size_t)dev.max_smem_optin - 2048 - 1024;  // static + alignment slack
   const int kb_total = (int)(K / kBK);
-  const int min_stages = pl.N < 128 ? 3 : 2;
+#ifndef FMLP_TC_NO_PAIR
+  pl.pair = pl.N >= 128;
+#endif
+  // per CTA: the pair kernel holds half of the B rows
+  const int b_rows = pl.pair ? pl.N / 2 : pl.N;
+  const int min_stages = (pl.N < 128 || pl.pair) ? 3 : 2;
   for (int ks = kTcMaxKs; ks >= 1; --ks) {
     if (ks > 1 && ks > kb_total) continue;
     pl.KS = ks;
     pl.a_bytes = ks * kATileBytes;
-    pl.b_bytes = ks * pl.N * kBK * 2;
+    pl.b_bytes = ks * b_rows * kBK * 2;
     pl.stage_bytes = (pl.a_bytes + pl.b_bytes + 1023) / 1024 * 1024;
     pl.stages = (int)std::min<size_t>(kMaxStages, budget / pl.stage_bytes);
     if (pl.stages >= min_stages) break;
@@ -747,23 +1149,47 @@ TcPlan make_tc_plan(int epi, int64_t M, int64_t K, const DeviceInfo& dev) {
   return pl;
 }
 
-cudaError_t allow_tc_smem(const DeviceInfo& dev) {
+template <typename Kernel>
+cudaError_t allow_tc_smem(Kernel kernel, const DeviceInfo& dev) {
   static std::mutex mu;
-  static std::set<int> done;
+  static std::set<std::pair<int, const void*>> done;
   std::lock_guard<std::mutex> lock(mu);
-  if (done.count(dev.device)) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(tc_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const auto key = std::make_pair(dev.device, (const void*)kernel);
+  if (done.count(key)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        dev.max_smem_optin - 2048);
-  if (e == cudaSuccess) done.insert(dev.device);
+  if (e == cudaSuccess) done.insert(key);
   return e;
+}
+
+// CTA pairs of tc_gemm_pair that can be resident at once (cluster placement
+// may leave some SMs unpaired), queried once per device.
+int pair_slots(const DeviceInfo& dev, size_t smem) {
+  static std::mutex mu;
+  static std::set<std::pair<int, int>> done;
+  static int slots[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev.device >= 0 && dev.device < 64 && slots[dev.device] > 0) return slots[dev.device];
+  int n = 0;
+  if (allow_tc_smem(tc_gemm_pair, dev) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(dev.sm_count & ~1));
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = smem;
+    if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_pair, &cfg) != cudaSuccess) n = 0;
+  }
+  if (n <= 0) n = dev.sm_count / 2;
+  n = std::min(n, dev.sm_count / 2);
+  if (dev.device >= 0 && dev.device < 64) slots[dev.device] = n;
+  return n;
 }
 
 cudaError_t launch_tc(const TcParams& p, const TcPlan& pl, const DeviceInfo& dev,
                       cudaStream_t stream) {
-  cudaError_t e = allow_tc_smem(dev);
+  cudaError_t e = pl.pair ? allow_tc_smem(tc_gemm_pair, dev) : allow_tc_smem(tc_gemm, dev);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.sched.ctas);
+  cfg.gridDim = dim3((unsigned)(pl.pair ? 2 * p.sched.ctas : p.sched.ctas));
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
@@ -772,7 +1198,7 @@ cudaError_t launch_tc(const TcParams& p, const TcPlan& pl, const DeviceInfo& dev
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, tc_gemm, p);
+  e = pl.pair ? cudaLaunchKernelEx(&cfg, tc_gemm_pair, p) : cudaLaunchKernelEx(&cfg, tc_gemm, p);
   if (e == cudaSuccess) note_launches(1);
   return e;
 }
@@ -795,9 +1221,11 @@ void fill_common(TcParams& p, const TcPlan& pl, int epi, int64_t M, int rows, in
   p.tmem_cols = pl.tmem_cols;
   p.sched.KB = (K / kBK + pl.KS - 1) / pl.KS;
   p.sched.ntok = pl.ntok;
-  p.sched.tiles = ((rows + kBM - 1) / kBM) * pl.ntok;
-  p.sched.ctas = (int)std::min<int64_t>(
-      {(int64_t)p.sched.tiles * p.sched.KB, (int64_t)dev.sm_count, (int64_t)kTcMaxCtas});
+  // work units are CTAs, or CTA pairs with 256-row tiles
+  const int tile_rows = pl.pair ? 2 * kBM : kBM;
+  p.sched.tiles = ((rows + tile_rows - 1) / tile_rows) * pl.ntok;
+  const int64_t units_max = pl.pair ? pair_slots(dev, pl.smem) : std::min(dev.sm_count, kTcMaxCtas);
+  p.sched.ctas = (int)std::min<int64_t>((int64_t)p.sched.tiles * p.sched.KB, units_max);
   // With one token tile no weight tile is reused, so plain stream-K balances
   // best.  Otherwise whole waves run data-parallel, and the stream-K rest is
   // kept at half a wave or more (folding one wave into it if needed) so that
@@ -825,7 +1253,8 @@ TcSizes tc_sizes(int64_t M, int64_t d, int64_t I, int sm_count) {
   z.partials = (size_t)sm_count * 2 * std::max(N_g, N_d) * kBM * 4;
   const int64_t tiles_g = ((2 * I + kBM - 1) / kBM) * ntok_g;
   const int64_t tiles_d = ((d + kBM - 1) / kBM) * ntok_d;
-  z.counters = (size_t)std::max(tiles_g, tiles_d) * 4;
+  // one counter per 128-row tile (per (256-row tile, rank) in the pair kernel)
+  z.counters = (size_t)(std::max(tiles_g, tiles_d) + 2) * 4;
   return z;
 }
 
@@ -863,7 +1292,8 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
                                            (uint64_t)d * 2, kBM, (uint32_t)pl.KS);
   if (e == cudaSuccess)
     e = encode_tmap_kblocks_bf16(&p.b_map, ws.b_hl, (uint64_t)pl.ntok * 2 * pl.Mt, (uint64_t)d,
-                                 (uint64_t)d * 2, (uint32_t)pl.N, (uint32_t)pl.KS);
+                                 (uint64_t)d * 2, (uint32_t)(pl.pair ? pl.N / 2 : pl.N),
+                                 (uint32_t)pl.KS);
   if (e != cudaSuccess) return e;
   fill_common(p, pl, kEpiSwiGLU, M, rows, (int)d, ws, dev);
   p.T = T;
@@ -902,7 +1332,7 @@ cudaError_t launch_tc_down(const void* a, int64_t M, const void* W_down, int64_t
                                            (uint64_t)I * 2, kBM, (uint32_t)pl.KS);
   if (e == cudaSuccess)
     e = encode_tmap_kblocks_bf16(&p.b_map, a, (uint64_t)M, (uint64_t)I, (uint64_t)I * 2,
-                                 (uint32_t)pl.N, (uint32_t)pl.KS);
+                                 (uint32_t)(pl.pair ? pl.N / 2 : pl.N), (uint32_t)pl.KS);
   if (e != cudaSuccess) return e;
   fill_common(p, pl, kEpiDown, M, (int)d, (int)I, ws, dev);
   p.I = (int)I;
