@@ -1119,22 +1119,23 @@ constexpr int kTcMaxKs = 4;
 // Stages of KS k-blocks.  On B200 one SM issues TMA copies at a few million
 // per second whatever their size (measured: ~2 M stages/s of two copies),
 // so a stage moves KS k-blocks of A and of B in one copy each.  KS is the
-// largest that still leaves a ring of 3 stages for narrow B operands (decode
-// batches: 8B M = 8 went from 3.2 to 5.4 TB/s, M = 32 gains 4% from 3 stages
-// of 3 k-blocks over 2 of 4) and of 2 stages for wide ones (verify, prefill:
-// deeper rings of single k-blocks were 6-13% slower there).
+// largest that still leaves a ring of min_stages stages: 3 for narrow B
+// operands (decode batches: 8B M = 8 went from 3.2 to 5.4 TB/s, M = 32
+// gains 4% from 3 stages of 3 k-blocks over 2 of 4) and 2 or 3 for wide ones
+// (below).
 TcPlan make_tc_plan(int epi, int64_t M, int64_t K, const DeviceInfo& dev) {
   TcPlan pl;
   tc_shape(epi, M, pl.Mt, pl.N, pl.C);
   pl.ntok = (int)((M + pl.Mt - 1) / pl.Mt);
   const size_t budget = (size_t)dev.max_smem_optin - 2048 - 1024;  // static + alignment slack
   const int kb_total = (int)(K / kBK);
-#ifndef FMLP_TC_NO_PAIR
+  // Two-SM tiles for wide operands (measured: pairing narrower ones, the
+  // M = 32 decode batch, was 4% slower).  Ring depth, measured per shape:
+  // streaming weights read once (one token tile: verify) want 3 stages of 2
+  // k-blocks; weight tiles reused from L2 (prefill) want 2 stages of 3.
   pl.pair = pl.N >= 128;
-#endif
-  // per CTA: the pair kernel holds half of the B rows
-  const int b_rows = pl.pair ? pl.N / 2 : pl.N;
-  const int min_stages = (pl.N < 128 || pl.pair) ? 3 : 2;
+  const int b_rows = pl.pair ? pl.N / 2 : pl.N;  // per CTA: a pair holds half the B rows
+  const int min_stages = pl.pair ? (pl.ntok > 1 ? 2 : 3) : (pl.N < 128 ? 3 : 2);
   for (int ks = kTcMaxKs; ks >= 1; --ks) {
     if (ks > 1 && ks > kb_total) continue;
     pl.KS = ks;
