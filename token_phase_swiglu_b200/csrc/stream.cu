@@ -143,7 +143,8 @@ struct Ring {
 
 struct CtaState {
   int abort;
-  int issued;  // stages issued by the producer
+  int issued;     // stages issued by the producer
+  int out_ready;  // fused_decode: 0 until every share of out is set, then 1 (-1: gave up)
 };
 
 __device__ __forceinline__ void init_ring(const Ring& r, CtaState& st) {
@@ -153,6 +154,7 @@ __device__ __forceinline__ void init_ring(const Ring& r, CtaState& st) {
   }
   st.abort = 0;
   st.issued = 0;
+  st.out_ready = 0;
   fence_barrier_init();
 }
 
@@ -704,6 +706,29 @@ __device__ bool consume_down_slice(Consumer& cs, const FusedParams& p, const flo
   return true;
 }
 
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+
+// Wait (one thread) for a shared-memory flag that another warp of the CTA
+// sets to nonzero; returns it, or 0 after limit_ns or when *abort is set.
+__device__ int wait_flag_cta(const int* flag, uint64_t limit_ns, volatile int* abort) {
+  int v = ld_acquire_cta(flag);
+  if (v) return v;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(32);
+    if ((v = ld_acquire_cta(flag)) != 0) return v;
+    if (*abort) return 0;
+    if (globaltimer_ns() - t0 > limit_ns) return 0;
+  }
+}
+
 // Wait (one thread) until the counter at `ctr` reaches `target`, with
 // acquire semantics, for at most limit_ns; false if it gave up.
 __device__ bool wait_counter(const uint32_t* ctr, uint32_t target, uint64_t limit_ns,
@@ -781,6 +806,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
       st.issued = pr.k;
     } else {
       init_out_share(p, mt, lane);
+      // Lane 1 then waits for every share of out and tells the consumers
+      // through shared memory, so that the L2 round trips of that wait stay
+      // off their path between the two phases.
+      if (lane == 1) {
+        int r = 1;
+        if (!wait_counter(p.inited, (uint32_t)p.n_init, p.ctl.wait_ns, &st.abort)) {
+          if (!st.abort) flag_timeout(&st, p.ctl.status);
+          r = -1;
+        }
+        st_release_cta(&st.out_ready, r);
+      }
     }
     __syncwarp();
   } else {
@@ -793,17 +829,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
     const bool ok = consume_gateup<MT>(cs, p.gu, g0, ng, s, rinv, nullptr, 0, mt, xch, slice,
                                        i0, p.swbox);
     // All of out must be set before anyone adds into it.  The shares are
-    // written at the start by CTAs already running, so by the end of the
-    // gate-up phase this normally returns at once (the ring keeps filling
-    // meanwhile).  The decision is published before the barrier so all
-    // consumer warps take it.
+    // written at the start by CTAs already running, and lane 1 of warp 0 has
+    // waited for them during the gate-up phase, so this normally reads its
+    // flag in shared memory at once.  The decision is published before the
+    // barrier so all consumer warps take it.
     if (ct == 0) {
       bool g = ok;
-      if (g && !wait_counter(p.inited, (uint32_t)p.n_init, p.ctl.wait_ns, &st.abort)) {
-        flag_timeout(&st, p.ctl.status);
-        g = false;
+      if (g) {
+        const int r = wait_flag_cta(&st.out_ready, p.ctl.wait_ns, &st.abort);
+        if (r == 0) flag_timeout(&st, p.ctl.status);
+        g = r == 1;
       }
-      __threadfence();
       go = g;
     }
     named_barrier_sync(kBarStage, kConsumers * 32);  // slice of a complete, out ready
