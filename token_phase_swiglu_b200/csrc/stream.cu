@@ -96,6 +96,18 @@ __device__ __forceinline__ uint64_t dot8bf(const uint4& w, const uint4& v, uint6
   return acc;
 }
 
+// Barrier `id` of all consumer warps; returns true if any of them failed.
+__device__ __forceinline__ bool consumer_barrier_any(int id, bool failed) {
+  uint32_t any;
+  asm volatile(
+      "{\n .reg .pred q, r;\n setp.ne.u32 q, %1, 0;\n"
+      " bar.red.or.pred r, %2, %3, q;\n selp.u32 %0, 1, 0, r;\n}"
+      : "=r"(any)
+      : "r"((uint32_t)failed), "r"(id), "n"(kConsumers * 32)
+      : "memory");
+  return any != 0;
+}
+
 // Per-group barrier of all consumer warps; returns true if any of them failed.
 __device__ __forceinline__ bool group_barrier_any(bool failed) {
   uint32_t any;
@@ -414,6 +426,79 @@ __device__ bool consume_gateup(Consumer& cs, const GateUpGeom& g, int g0, int n_
     }
   }
   return true;
+}
+
+// fused_decode's gate-up consumer: as consume_gateup, but each warp leaves
+// its warp-reduced gate and up sums of every group in `part` (shared memory,
+// [group][pair][half][gate, up][MT]) instead of combining the column halves
+// group by group, so that the warps meet at no barrier during the phase and
+// can run up to a ring's depth apart.  finish_slice combines them.
+template <int MT>
+__device__ bool consume_gateup_parts(Consumer& cs, const GateUpGeom& g, int n_groups,
+                                     const float* s, float* part) {
+  const int c = (threadIdx.x >> 5) - 1, lane = cs.lane;
+  const int pr = c & (kGroup - 1), half = c / kGroup;
+  for (int j = 0; j < n_groups; ++j) {
+    uint64_t ag[2][MT], au[2][MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) ag[0][m] = ag[1][m] = au[0][m] = au[1][m] = 0ull;
+    for (int ch = 0; ch < g.nchunks; ++ch) {
+      const uint8_t* buf = cs.wait_full();
+      if (!buf) return false;
+      const int k0 = ch * g.kc;
+      const int nv = min(g.kc, g.d - k0) / 8;
+      const uint8_t* bg = buf + (size_t)pr * g.kc * 2;
+      const uint8_t* bu = buf + (size_t)(kGroup + pr) * g.kc * 2;
+      const int kv0 = k0 / 8;
+      for (int v = lane + 32 * half; v < nv; v += 128) {  // vectors v and v + 64
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int vv = v + 64 * h;
+          if (h == 0 || vv < nv) {
+            const uint4 wg = lds128(bg + 16 * vv);
+            const uint4 wu = lds128(bu + 16 * vv);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              const float4* sp = reinterpret_cast<const float4*>(s + (int64_t)m * g.d) + kv0 + vv;
+              const float4 s0 = sp[0], s1 = sp[g.d / 8];
+              ag[h][m] = dot8(wg, s0, s1, ag[h][m]);
+              au[h][m] = dot8(wu, s0, s1, au[h][m]);
+            }
+          }
+        }
+      }
+      cs.release();
+    }
+    float* dst = part + ((j * kGroup + pr) * 2 + half) * 2 * MT;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const float gs = warp_sum(hsum2(ag[0][m]) + hsum2(ag[1][m]));
+      const float us = warp_sum(hsum2(au[0][m]) + hsum2(au[1][m]));
+      if (lane == 0) {
+        dst[m] = gs;
+        dst[MT + m] = us;
+      }
+    }
+  }
+  return true;
+}
+
+// a = bf16(SiLU(r g) * r u) for the CTA's w = 4 * n_groups pairs, from the
+// halves' sums in `part`, into slice[m * ld + i] (as f32; rows >= mt zero).
+// All consumer threads, after a barrier that follows consume_gateup_parts.
+template <int MT>
+__device__ void finish_slice(const float* part, int n_groups, const float* rinv, int mt,
+                             float* slice, int ld) {
+  const int ct = threadIdx.x - 32;
+  for (int i = ct; i < n_groups * kGroup; i += kConsumers * 32) {
+    const float* q = part + i * 4 * MT;  // [half 0: g, u][half 1: g, u]
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const float gt = q[m] + q[2 * MT + m], ut = q[MT + m] + q[3 * MT + m];
+      const __nv_bfloat16 av = __float2bfloat16_rn(silu_mul(gt * rinv[m], ut * rinv[m]));
+      slice[m * ld + i] = m < mt ? __bfloat162float(av) : 0.f;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -774,17 +859,16 @@ template <int MT>
 __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constant__ FusedParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ float red[kConsumers][MT];
-  __shared__ float xch[2 * kGroup * 2 * MT];
   __shared__ CtaState st;
-  __shared__ int go;
 
   Ring ring;
   ring.full = reinterpret_cast<uint64_t*>(smem);
   ring.empty = ring.full + kMaxStages;
   float* s = reinterpret_cast<float*>(smem + kHeader);                          // [MT][d]
   float* slice = reinterpret_cast<float*>(smem + kHeader + align128((size_t)MT * p.d * 4));
+  float* part = slice + align128((size_t)MT * p.swbox * 4) / 4;  // [swbox / 4][kGroup][2][2][MT]
   ring.stage0 = smem + kHeader + align128((size_t)MT * p.d * 4) +
-                align128((size_t)MT * p.swbox * 4);
+                align128((size_t)MT * p.swbox * 4) + align128((size_t)MT * p.swbox * 16);
   ring.stages = p.stages;
   ring.stage_bytes = p.stage_bytes;
 
@@ -826,24 +910,23 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
     Consumer cs{ring, &st, p.ctl, 0, lane};
     float rinv[MT];
     stage_x_gamma<MT>(p.x, nullptr, p.eps, p.d, 0, mt, s, red, rinv);
-    const bool ok = consume_gateup<MT>(cs, p.gu, g0, ng, s, rinv, nullptr, 0, mt, xch, slice,
-                                       i0, p.swbox);
+    bool ok = consume_gateup_parts<MT>(cs, p.gu, ng, s, part);
     // All of out must be set before anyone adds into it.  The shares are
     // written at the start by CTAs already running, and lane 1 of warp 0 has
     // waited for them during the gate-up phase, so this normally reads its
-    // flag in shared memory at once.  The decision is published before the
-    // barrier so all consumer warps take it.
-    if (ct == 0) {
-      bool g = ok;
-      if (g) {
-        const int r = wait_flag_cta(&st.out_ready, p.ctl.wait_ns, &st.abort);
-        if (r == 0) flag_timeout(&st, p.ctl.status);
-        g = r == 1;
-      }
-      go = g;
+    // flag in shared memory at once.
+    if (ct == 0 && ok) {
+      const int r = wait_flag_cta(&st.out_ready, p.ctl.wait_ns, &st.abort);
+      if (r == 0) flag_timeout(&st, p.ctl.status);
+      ok = r == 1;
     }
-    named_barrier_sync(kBarStage, kConsumers * 32);  // slice of a complete, out ready
-    if (go) consume_down_slice<MT>(cs, p, slice, w, mt);
+    // Every warp's sums are in `part` and out is ready, or someone gave up:
+    // all consumer warps take the same decision.
+    if (!consumer_barrier_any(kBarStage, !ok)) {
+      finish_slice<MT>(part, ng, rinv, mt, slice, p.swbox);
+      named_barrier_sync(kBarStage, kConsumers * 32);  // slice of a complete
+      consume_down_slice<MT>(cs, p, slice, w, mt);
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -1039,7 +1122,9 @@ FusedPlan make_fused_plan(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev
   f.rows_d = f.swbox <= 128 ? 256 : 128;
   f.nrb = (int)((d + f.rows_d - 1) / f.rows_d);
   const size_t down_stage = align128((size_t)f.swbox * f.rows_d * 2);
-  const size_t act = align128((size_t)M * d * 4) + align128((size_t)M * f.swbox * 4);
+  // s (x * gamma), the slice of a, and the halves' gate/up sums
+  const size_t act = align128((size_t)M * d * 4) + align128((size_t)M * f.swbox * 4) +
+                     align128((size_t)M * f.swbox * 16);
   if (kHeader + act >= budget) return FusedPlan();
   for (int64_t target = kMaxStageBytes; target >= 4096; target /= 2) {
     const Chunking gu = chunk_rows(d, kGateRows, target);
