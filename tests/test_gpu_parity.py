@@ -410,6 +410,18 @@ def test_fused_and_two_kernel_paths_agree(fm):
         assert norm <= 1e-5, norm
 
 
+def test_fused_decode_with_shorter_down_stages(fm):
+    """8B-shaped batch of 4 rows: with 256-row W_down stages the fused kernel's
+    ring would have under three slots, so its W_down stages hold as many rows
+    as a gate-up stage's bytes (152 here).  Still one launch per call."""
+    p = wl.make_problem(4, 4096, 14336, sigma=0.02, seed=5, residual=True)
+    n0 = fm.fmlp_kernel_launch_count()
+    got = run_forward(fm, p, T=16, residual=True)
+    assert fm.fmlp_kernel_launch_count() - n0 == 2  # pack + one fused forward
+    assert_parity(got, oracle_out(p, residual=True), oracle_out(p, residual=True,
+                                                               intermediate="bf16"))
+
+
 @pytest.mark.parametrize("M,d,I", [(1, 32768, 64), (4, 32768, 64), (1, 64, 65536), (3, 64, 65536),
                                    (2, 8, 8)])
 def test_maximum_and_minimum_sizes(fm, M, d, I):

@@ -711,7 +711,8 @@ struct FusedParams {
   int M, d, I;
   int units;           // I / 8: slices are cut at multiples of 8 pairs (16-byte columns)
   int swbox;           // W_down slice box width (>= every CTA's slice, odd multiple of 8)
-  int rows_d;          // W_down rows per stage (256, or 128 for wide slices)
+  int rows_d;          // W_down rows per stage (256, or 128 for wide slices; fewer if
+                       // the ring would have under three slots)
   int nrb;             // row blocks = ceil(d / rows_d)
   int stages, stage_bytes;
 };
@@ -729,15 +730,16 @@ __device__ void produce_down_slice(Producer& pr, const FusedParams& p, int i0) {
 }
 
 // Each consumer thread owns one W_down row of the stage (two threads per row,
-// column halves, when rows_d == 128) and adds its partial dot products with
-// the CTA's slice of a into acc.
+// column halves, for slices wider than 128 columns) and adds its partial dot
+// products with the CTA's slice of a into out.
 template <int MT>
 __device__ bool consume_down_slice(Consumer& cs, const FusedParams& p, const float* slice,
                                    int w, int mt) {
   const int ct = threadIdx.x - 32;
-  const int r = p.rows_d == 256 ? ct : (ct & 127);
+  const bool halves = p.swbox > 128;
+  const int r = halves ? (ct & 127) : ct;
   int c0 = 0, c1 = w;
-  if (p.rows_d != 256) {
+  if (halves) {
     const int hw = ((w / 2) + 7) / 8 * 8;
     if (ct < 128) c1 = hw; else c0 = hw;
   }
@@ -745,7 +747,7 @@ __device__ bool consume_down_slice(Consumer& cs, const FusedParams& p, const flo
     const uint8_t* buf = cs.wait_full();
     if (!buf) return false;
     const int n = rb * p.rows_d + r;
-    if (n < p.d) {
+    if (r < p.rows_d && n < p.d) {
       const uint8_t* row = buf + (size_t)r * p.swbox * 2;
       float acc[2][MT];
 #pragma unroll
@@ -1119,18 +1121,26 @@ FusedPlan make_fused_plan(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev
   int sw_units = max_units | 1;  // odd count of 16-byte columns: conflict-free row reads
   f.swbox = 8 * sw_units;
   if (f.swbox > 256) return FusedPlan();
-  f.rows_d = f.swbox <= 128 ? 256 : 128;
-  f.nrb = (int)((d + f.rows_d - 1) / f.rows_d);
-  const size_t down_stage = align128((size_t)f.swbox * f.rows_d * 2);
+  const int full_rows = f.swbox <= 128 ? 256 : 128;
+  const size_t down_stage = align128((size_t)f.swbox * full_rows * 2);
   // s (x * gamma), the slice of a, and the halves' gate/up sums
   const size_t act = align128((size_t)M * d * 4) + align128((size_t)M * f.swbox * 4) +
                      align128((size_t)M * f.swbox * 16);
   if (kHeader + act >= budget) return FusedPlan();
   for (int64_t target = kMaxStageBytes; target >= 4096; target /= 2) {
     const Chunking gu = chunk_rows(d, kGateRows, target);
-    const size_t slot = std::max<size_t>(gu.stage_bytes, down_stage);
+    // W_down stages of full_rows rows, or, if the ring would then have under
+    // three slots, of as many rows as a gate-up stage's bytes hold
+    size_t slot = std::max<size_t>(gu.stage_bytes, down_stage);
+    f.rows_d = full_rows;
+    if ((budget - kHeader - act) / slot < 3) {
+      slot = gu.stage_bytes;
+      f.rows_d = std::min(full_rows, (int)(slot / (f.swbox * 2)) / 8 * 8);
+      if (f.rows_d < 128) continue;  // too many small copies: leave it to the other paths
+    }
     const size_t fit = (budget - kHeader - act) / slot;
     if (fit < 3) continue;
+    f.nrb = (int)((d + f.rows_d - 1) / f.rows_d);
     f.gu = gu;
     f.mt = (int)M;
     f.stage_bytes = (int)slot;
