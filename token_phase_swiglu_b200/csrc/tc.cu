@@ -248,7 +248,9 @@ struct TcShared {
   uint32_t tmem_base;
   int abort;
   int last;
+  int head_done;       // the other contributor of this CTA's last gate-up tile has arrived
   int k_issued;        // stages issued by the producer
+  float rinv_s[2][kBM];  // 1/RMS of the token tile of each accumulator buffer (SwiGLU)
 };
 
 __device__ __forceinline__ void tc_flag(TcShared* sh, uint32_t* status) {
@@ -258,9 +260,11 @@ __device__ __forceinline__ void tc_flag(TcShared* sh, uint32_t* status) {
 
 // SwiGLU epilogue of CW logical columns [col0, col0 + CW) of one finished
 // gate-up tile (warps 2-5; vals[j] = D[row, col0 + j], hi + lo summed).
+// rv: 1/RMS of the token tile's rows (shared memory).
 template <int CW>
 __device__ __forceinline__ void epilogue_columns(const TcParams& p, int tt, int row,
-                                                 const float (&vals)[CW], int col0) {
+                                                 const float (&vals)[CW], int col0,
+                                                 const float* rv) {
   // SwiGLU: within a 2T-row interleave tile rows [0,T) are gate, [T,2T) up;
   // the partner row is lane ^ T (T in {8, 16}).  The gate lane finishes the
   // first half of the chunk's tokens, the up lane the second half.
@@ -276,13 +280,13 @@ __device__ __forceinline__ void epilogue_columns(const TcParams& p, int tt, int 
     u[j] = is_gate ? recv : vals[H + j];
   }
   const int pair = (row / (2 * T)) * T + (row % T);
-  const int tok0 = tt * p.Mt + col0 + (is_gate ? 0 : H);
+  const int loc0 = col0 + (is_gate ? 0 : H), tok0 = tt * p.Mt + loc0;
   if (row < p.rows && pair < p.I) {
 #pragma unroll
     for (int j = 0; j < H; ++j) {
       const int m = tok0 + j;
       if (m < p.M) {
-        const float r = p.rinv[m];
+        const float r = rv[loc0 + j];
         p.a_out[(int64_t)m * p.I + pair] = __float2bfloat16_rn(silu_mul(g[j] * r, u[j] * r));
       }
     }
@@ -309,20 +313,17 @@ __device__ __forceinline__ void tile_cols(const TcParams& p, uint32_t tb, int co
 // contributors' partials, CW logical columns at a time, then the epilogue.
 template <int CW>
 __device__ void finish_tile(const TcParams& p, int t, uint32_t tb, bool whole, int c_first,
-                            int c_last, int r_local) {
+                            int c_last, int r_local, const float* rv) {
   const int ncol = p.epi == kEpiSwiGLU ? p.Mt : p.N;
   const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
   const int row = rt * kBM + r_local;
   for (int c0 = 0; c0 < ncol; c0 += CW) {
     float vals[CW];
-    tile_cols<CW>(p, tb, c0, vals);
-    if (p.epi == kEpiSwiGLU) {
-      float lo[CW];
-      tile_cols<CW>(p, tb, p.Mt + c0, lo);  // lo half of x*gamma
 #pragma unroll
-      for (int j = 0; j < CW; ++j) vals[j] += lo[j];
-    }
+    for (int j = 0; j < CW; ++j) vals[j] = 0.f;
     if (!whole) {
+      // the other contributors' partials first: their L2 round trip
+      // overlaps the accumulator reads below
       for (int cc = c_first; cc <= c_last; ++cc) {
         if (cc == (int)blockIdx.x) continue;
         int64_t cu0, cu1;
@@ -336,7 +337,16 @@ __device__ void finish_tile(const TcParams& p, int t, uint32_t tb, bool whole, i
         }
       }
     }
-    epilogue_columns<CW>(p, tt, row, vals, c0);
+    float acc[CW];
+    tile_cols<CW>(p, tb, c0, acc);
+#pragma unroll
+    for (int j = 0; j < CW; ++j) vals[j] += acc[j];
+    if (p.epi == kEpiSwiGLU) {
+      tile_cols<CW>(p, tb, p.Mt + c0, acc);  // lo half of x*gamma
+#pragma unroll
+      for (int j = 0; j < CW; ++j) vals[j] += acc[j];
+    }
+    epilogue_columns<CW>(p, tt, row, vals, c0, rv);
   }
 }
 
@@ -524,10 +534,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
       int t, kb0, kb1;
       segment(p.sched, u0, u1, s, t, kb0, kb1);
       const int buf = s & 1;
+      // A gate-up tile shared by two CTAs: the one holding its first
+      // k-blocks reaches it at the end of its range, long after the other
+      // (whose range starts inside it) has stored its partial.  Look at the
+      // tile's counter while the MMAs still run: if the other contributor has
+      // arrived, this CTA finishes the tile without storing a partial of its
+      // own or taking part in the count (the other one has left it).
+      bool head_only = false;
+      if (p.epi == kEpiSwiGLU && !(kb0 == 0 && kb1 == p.sched.KB) && kb0 == 0) {
+        const int64_t tu = (int64_t)(t - p.sched.sk_tile0()) * p.sched.KB;
+        if (p.sched.cta_of(tu + p.sched.KB - 1) == (int)blockIdx.x + 1) {
+          if (et == 0) sh.head_done = ld_acquire_gpu(p.counters + t) == 1u;
+          head_only = true;
+        }
+      }
+      if (p.epi == kEpiSwiGLU) {  // 1/RMS of the token tile, while the MMAs run
+        const int tt = t % p.sched.ntok;
+        for (int i = et; i < p.Mt; i += 128) {
+          const int m = tt * p.Mt + i;
+          sh.rinv_s[buf][i] = m < p.M ? __ldg(p.rinv + m) : 0.f;
+        }
+      }
       const bool got =
           mbar_wait_bounded(&sh.acc_full[buf], (uint32_t)((s >> 1) & 1), p.wait_ns, abort);
       if (!got && lane == 0) tc_flag(&sh, p.status);
-      if (epilogue_barrier_any(!got)) break;
+      if (epilogue_barrier_any(!got)) break;  // also publishes sh.head_done and sh.rinv_s
       tc_fence_after();
       const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.C * p.N);
       if (p.epi == kEpiDown) {
@@ -546,7 +577,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
       const int c_first = whole ? 0 : p.sched.cta_of(tu);
       const int c_last = whole ? 0 : p.sched.cta_of(tu + p.sched.KB - 1);
       bool finalize = whole;
-      if (!whole) {
+      if (head_only && sh.head_done) {
+        // the other contributor's partial is visible (acquire above)
+        finalize = true;
+      } else if (!whole) {
         // this CTA's partial (chains summed): slot 0 if the tile is where its
         // range starts, else 1.  N is a multiple of 16.
         const int slot = (t == p.sched.sk_tile0() + (int)(u0 / p.sched.KB)) ? 0 : 1;
@@ -573,9 +607,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm(const __grid_constant__
       }
       if (finalize) {
         // a chunk width that divides the logical columns (a multiple of 8)
-        if (ncol % 32 == 0) finish_tile<32>(p, t, tb, whole, c_first, c_last, r_local);
-        else if (ncol % 16 == 0) finish_tile<16>(p, t, tb, whole, c_first, c_last, r_local);
-        else finish_tile<8>(p, t, tb, whole, c_first, c_last, r_local);
+        const float* rv = sh.rinv_s[buf];
+        if (ncol % 32 == 0) finish_tile<32>(p, t, tb, whole, c_first, c_last, r_local, rv);
+        else if (ncol % 16 == 0) finish_tile<16>(p, t, tb, whole, c_first, c_last, r_local, rv);
+        else finish_tile<8>(p, t, tb, whole, c_first, c_last, r_local, rv);
         if (!whole && et == 0) atomicExch(p.counters + t, 0u);
       }
       tc_fence_before();
@@ -700,7 +735,7 @@ __device__ __forceinline__ bool segment_of(const Sched& S, int me, int64_t u0, i
 // accumulator plus the other pairs' partials of the same rank.
 template <int CW>
 __device__ void finish_tile_pair(const TcParams& p, int t, int rank, uint32_t tb, bool whole,
-                                 int c_first, int c_last, int me, int r_local) {
+                                 int c_first, int c_last, int me, int r_local, const float* rv) {
   const int ncol = p.Mt;
   const int rt = t / p.sched.ntok, tt = t % p.sched.ntok;
   const int row = rt * 2 * kBM + rank * kBM + r_local;
@@ -725,7 +760,7 @@ __device__ void finish_tile_pair(const TcParams& p, int t, int rank, uint32_t tb
                      __ldcg(part + (size_t)(p.Mt + c0 + j) * kBM + r_local);
       }
     }
-    epilogue_columns<CW>(p, tt, row, vals, c0);
+    epilogue_columns<CW>(p, tt, row, vals, c0, rv);
   }
 }
 
@@ -917,10 +952,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       int t, kb0, kb1;
       segment_of(p.sched, me, u0, u1, s, t, kb0, kb1);
       const int buf = s & 1;
+      if (p.epi == kEpiSwiGLU) {  // 1/RMS of the token tile, while the MMAs run
+        const int tt = t % p.sched.ntok;
+        for (int i = et; i < p.Mt; i += 128) {
+          const int m = tt * p.Mt + i;
+          sh.rinv_s[buf][i] = m < p.M ? __ldg(p.rinv + m) : 0.f;
+        }
+      }
       const bool got =
           mbar_wait_bounded(&sh.acc_full[buf], (uint32_t)((s >> 1) & 1), p.wait_ns, abort);
       if (!got && lane == 0) tc_flag(&sh, p.status);
-      if (epilogue_barrier_any(!got)) break;
+      if (epilogue_barrier_any(!got)) break;  // also publishes sh.rinv_s
       tc_fence_after();
       const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * p.C * N);
       if (p.epi == kEpiDown) {
@@ -957,12 +999,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
           if (finalize) __threadfence();
         }
         if (finalize) {
+          const float* rv = sh.rinv_s[buf];
           if (ncol % 32 == 0)
-            finish_tile_pair<32>(p, t, rank, tb, whole, c_first, c_last, me, r_local);
+            finish_tile_pair<32>(p, t, rank, tb, whole, c_first, c_last, me, r_local, rv);
           else if (ncol % 16 == 0)
-            finish_tile_pair<16>(p, t, rank, tb, whole, c_first, c_last, me, r_local);
+            finish_tile_pair<16>(p, t, rank, tb, whole, c_first, c_last, me, r_local, rv);
           else
-            finish_tile_pair<8>(p, t, rank, tb, whole, c_first, c_last, me, r_local);
+            finish_tile_pair<8>(p, t, rank, tb, whole, c_first, c_last, me, r_local, rv);
           if (!whole && et == 0) atomicExch(p.counters + 2 * t + rank, 0u);
         }
       }
@@ -1010,12 +1053,6 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
   // The GEMM launched next may start (and prefetch its weights) right away;
   // it waits for this grid's completion before it reads what this writes.
   grid_launch_dependents();
-  grid_dependency_wait();
-  // The stream-K arrival counters start every call at zero, whatever a
-  // previous call (an aborted one, or one of another shape) left there.  The
-  // previous call's kernels are complete once the wait above returns.
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < ncounters; i += gridDim.x * blockDim.x)
-    counters[i] = 0u;
   const int slot = blockIdx.x;
   const int j = slot / Mt, i = slot % Mt;
   const int m = slot;
@@ -1023,10 +1060,9 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
   __nv_bfloat16* lo = hi + (int64_t)Mt * d;
   __shared__ float red[8];
   float ss = 0.f;
-  for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
-    uint4 xv = make_uint4(0, 0, 0, 0);
-    if (m < M) xv = ld_keep(x + (int64_t)m * d + (int64_t)v * 8);
-    const uint4 gv = ld_keep(gamma + (int64_t)v * 8);
+  // x * gamma, split into hi + lo, and the sum of squares of the row, for 8
+  // columns [8v, 8v + 8) given x and gamma there
+  auto split8 = [&](int v, const uint4& xv, const uint4& gv) {
     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
     uint32_t hw[4], lw[4];
 #pragma unroll
@@ -1043,7 +1079,43 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
     }
     reinterpret_cast<uint4*>(hi)[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     reinterpret_cast<uint4*>(lo)[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  };
+  const int nv = d / 8;
+  constexpr int kRegV = 4;  // vectors per thread held in registers (d <= 8192 at 256 threads)
+  if (nv <= kRegV * (int)blockDim.x) {
+    // gamma (a weight) before the dependency wait; every x load of the
+    // thread in flight at once after it
+    uint4 gv[kRegV], xv[kRegV];
+#pragma unroll
+    for (int q = 0; q < kRegV; ++q) {
+      const int v = threadIdx.x + q * blockDim.x;
+      gv[q] = v < nv ? ld_keep(gamma + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
+    }
+    grid_dependency_wait();
+#pragma unroll
+    for (int q = 0; q < kRegV; ++q) {
+      const int v = threadIdx.x + q * blockDim.x;
+      xv[q] = make_uint4(0, 0, 0, 0);
+      if (m < M && v < nv) xv[q] = ld_keep(x + (int64_t)m * d + (int64_t)v * 8);
+    }
+#pragma unroll
+    for (int q = 0; q < kRegV; ++q) {
+      const int v = threadIdx.x + q * blockDim.x;
+      if (v < nv) split8(v, xv[q], gv[q]);
+    }
+  } else {
+    grid_dependency_wait();
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      uint4 xv = make_uint4(0, 0, 0, 0);
+      if (m < M) xv = ld_keep(x + (int64_t)m * d + (int64_t)v * 8);
+      split8(v, xv, ld_keep(gamma + (int64_t)v * 8));
+    }
   }
+  // The stream-K arrival counters start every call at zero, whatever a
+  // previous call (an aborted one, or one of another shape) left there.  The
+  // previous call's kernels are complete once the wait above returns.
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < ncounters; c += gridDim.x * blockDim.x)
+    counters[c] = 0u;
   // The down GEMM adds its split-K shares into out: start it at the residual
   // (or zero), one token row per CTA.
   if (out && m < M)
