@@ -459,6 +459,30 @@ def test_tensor_core_path(fm, M, d, I, T, residual):
     assert_parity(got, ref, oracle_out(p, residual=residual, intermediate="bf16"))
 
 
+@pytest.mark.parametrize("M,d,I", [(24, 512, 1024), (72, 256, 512)])
+def test_tensor_core_back_to_back_calls(fm, M, d, I):
+    """Many calls queued on one stream with one workspace and no sync between
+    them, alternating with and without residual.  These grids leave SMs free,
+    so each kernel's weight prefetch runs beside the previous kernel; the
+    next call's prologue resets the counters and out.  Every output must
+    still match the oracle."""
+    dev = torch.device("cuda:0")
+    p = wl.make_problem(M, d, I, sigma=0.03, seed=17, residual=True)
+    g = {k: v.to(dev) for k, v in p.items()}
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(g["W_gate"], g["W_up"], 16, packed)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    outs = [torch.full((M, d), float("nan"), dtype=torch.float32, device=dev) for _ in range(24)]
+    for i, out in enumerate(outs):
+        fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, 16, g["W_down"], out, ws,
+                        residual=g["residual"] if i % 2 else None)
+    torch.cuda.synchronize()
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+    refs = [oracle_out(p, residual=False), oracle_out(p, residual=True)]
+    for i, out in enumerate(outs):
+        assert_parity(out.cpu().double().numpy(), refs[i % 2])
+
+
 @pytest.mark.parametrize("M,d,I", [(24, 512, 1024), (130, 384, 640)])
 def test_tensor_core_down_proj_alone(fm, M, d, I):
     """fmlp_down_proj on the tensor path sets out to the residual (or zero)

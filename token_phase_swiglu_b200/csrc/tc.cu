@@ -258,6 +258,18 @@ __device__ __forceinline__ void tc_flag(TcShared* sh, uint32_t* status) {
   atomicOr(status, kStatusTimeout);
 }
 
+// SiLU(g) * u with the hardware exp2 and reciprocal approximations.  Their
+// relative error (a few 1e-7) is far below the bf16 rounding of a that
+// follows (2^-9), and the exact form's limits hold: for g << 0, exp(-g) is
+// +inf, its reciprocal 0 and the result -0 * u; for g >> 0 it is g * u.  The
+// epilogue runs one warp per scheduler, so the exact division and exp would
+// sit on the tail of every gate-up GEMM.
+__device__ __forceinline__ float silu_mul_fast(float g, float u) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + __expf(-g)));
+  return g * r * u;
+}
+
 // SwiGLU epilogue of CW logical columns [col0, col0 + CW) of one finished
 // gate-up tile (warps 2-5; vals[j] = D[row, col0 + j], hi + lo summed).
 // rv: 1/RMS of the token tile's rows (shared memory).
@@ -287,7 +299,7 @@ __device__ __forceinline__ void epilogue_columns(const TcParams& p, int tt, int 
       const int m = tok0 + j;
       if (m < p.M) {
         const float r = rv[loc0 + j];
-        p.a_out[(int64_t)m * p.I + pair] = __float2bfloat16_rn(silu_mul(g[j] * r, u[j] * r));
+        p.a_out[(int64_t)m * p.I + pair] = __float2bfloat16_rn(silu_mul_fast(g[j] * r, u[j] * r));
       }
     }
   }
