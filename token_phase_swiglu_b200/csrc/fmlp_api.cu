@@ -29,9 +29,16 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }  // N
 
 inline uint32_t* status_word(void* workspace) { return (uint32_t*)workspace; }
 
-// The tensor-core path takes token counts above the fused decode kernel's range.
+// The tensor-core path takes token counts above the fused decode kernel's
+// range, and from 2 rows on where it is the faster one.  The fused kernel's
+// CUDA-core consumers do M dot products per weight and fall behind HBM after
+// a row or two; the tensor-core path pays about 10 us per layer for its three
+// launches whatever M.  Measured per layer on B200 (fused / tensor-core):
+// Phi-3-shaped (151 MB of weights) M=2 28.3 / 36.9 us, M=3 33.8 / 37.1,
+// M=4 39.7 / 37.0; 8B-shaped (352 MB) M=2 63.7 / 60.4, M=3 72.4 / 61.4.
 bool use_tc(int64_t M, int64_t d, int64_t I, int T) {
-  return M > kFusedMaxM && tc_supported(M, d, I, T);
+  if (M < 2 || !tc_supported(M, d, I, T)) return false;
+  return M > kFusedMaxM || M >= 4 || 6 * d * I > (int64_t)200000000;
 }
 
 TcWorkspace tc_workspace(void* workspace, const WorkspaceLayout& L) {
@@ -111,7 +118,7 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
   L.zero_end = off;
   L.a = off;
   off += align256((size_t)M * (size_t)I * 2);
-  if (M > kFusedMaxM && tc_supported(M, d, I, 16)) {  // the tensor-core path may run
+  if (M >= 2 && tc_supported(M, d, I, 16)) {  // the tensor-core path may run
     const TcSizes z = tc_sizes(M, d, I, kTcMaxCtas);
     L.b_hl = off;
     off += align256(z.b_hl);
@@ -258,7 +265,7 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
   uint32_t* status = status_word(workspace);
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
-  if (fused_decode_supported(M, d, I, *dev)) {
+  if (!use_tc(M, d, I, tile_T) && fused_decode_supported(M, d, I, *dev)) {
     uint32_t* ticket = (uint32_t*)((char*)workspace + L.ticket);
     uint32_t* inited = (uint32_t*)((char*)workspace + L.inited);
     uint32_t* done = (uint32_t*)((char*)workspace + L.done);
