@@ -105,8 +105,9 @@ FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
  *
  * Precision: x*gamma is formed exactly in f32 and the contraction keeps it at
  * f32 precision (CUDA-core path) or as an exact hi+lo bf16 pair (tensor-core
- * path); accumulation is f32; a is rounded once to bf16 (round to nearest
- * even); out is f32.  out is written by several thread blocks adding into it
+ * path); accumulation is f32; SiLU is evaluated in f32 (on the tensor-core
+ * path with the hardware exp2 and reciprocal approximations, relative error
+ * about 1e-6); a is rounded once to bf16 (round to nearest even); out is f32.  out is written by several thread blocks adding into it
  * (f32 atomics), so the summation order, and the last bits of out, may differ
  * from run to run.  out must not overlap any input.
  *
