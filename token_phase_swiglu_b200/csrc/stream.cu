@@ -13,17 +13,19 @@
 //     large copies (up to 64 KB): on B200 a bulk-copy ring is limited by the
 //     number of copies per second far more than by the bytes in flight, so
 //     copies are made as large as the rows allow;
-//   * four consumer warps share every stage: warp w owns gate/up pair w (or
-//     W_down row w) of the group, dots it with the activations held in shared
-//     memory, and arrives on the stage's "empty" mbarrier;
+//   * eight consumer warps share every stage: warp w owns gate/up pair w & 3
+//     (or W_down row w & 3) of the group and column half w >> 2, dots it with
+//     the activations held in shared memory, leaves its sums in shared memory
+//     and arrives on the stage's "empty" mbarrier; the halves are combined
+//     once, after the phase;
 //   * fused_decode runs both steps in one launch, the "Fusion MLP" of the
 //     pages.  CTA b owns a slice of the intermediate dimension: it streams the
 //     gate/up rows of its pairs, keeps its slice of a (rounded to bf16) in
 //     shared memory, then streams the matching column slice of W_down (2-D
-//     TMA tiles of 256 rows) and adds its partial down projection into an f32
-//     accumulator in the workspace (red.global.add).  The last CTA to finish
-//     adds the residual, writes out and re-zeroes the accumulator.  No CTA
-//     waits for another, and `a` never travels through global memory;
+//     TMA tiles of 256 rows) and adds its partial down projection straight
+//     into out (red.global.add), which the first CTAs to arrive have set to
+//     the residual (or zero).  No CTA waits for another CTA's results, and
+//     `a` never travels through global memory;
 //   * launches use programmatic dependent launch: a kernel's producer starts
 //     streaming weights before the previous kernel on the stream has
 //     finished; only the consumers wait for its results.
@@ -52,7 +54,6 @@ constexpr uint64_t kDrainNs = 1000000000ull;      // in-flight copies land long 
 constexpr int kGateRows = 2 * kGroup;             // rows per gate-up stage (4 gate + 4 up)
 constexpr int kDownRows = kGroup;                 // rows per down stage
 constexpr int kBarStage = 1;                      // named barrier: consumer-only sync
-constexpr int kBarGroup = 2;                      // named barrier: per-group combine
 
 static_assert(2 * kMaxStages * 8 <= kHeader, "barrier block overflows its header");
 
@@ -108,17 +109,6 @@ __device__ __forceinline__ bool consumer_barrier_any(int id, bool failed) {
   return any != 0;
 }
 
-// Per-group barrier of all consumer warps; returns true if any of them failed.
-__device__ __forceinline__ bool group_barrier_any(bool failed) {
-  uint32_t any;
-  asm volatile(
-      "{\n .reg .pred q, r;\n setp.ne.u32 q, %1, 0;\n"
-      " bar.red.or.pred r, %2, %3, q;\n selp.u32 %0, 1, 0, r;\n}"
-      : "=r"(any)
-      : "r"((uint32_t)failed), "n"(kBarGroup), "n"(kConsumers * 32)
-      : "memory");
-  return any != 0;
-}
 
 // Packed-row index of gate row i (its up row is T rows further on).
 __device__ __forceinline__ int64_t gate_row(int i, int T) {
@@ -350,89 +340,15 @@ __device__ void stage_x_gamma(const __nv_bfloat16* x, const __nv_bfloat16* gamma
   }
 }
 
-// Consumer warps: pair w & 3 of every group, column half w >> 2; writes a[m, i].
-// xch: [2][kGroup][2*MT] floats of shared memory for the halves' partial sums.
-// If `slice` is given, a goes to shared memory instead: slice[m * slice_ld +
-// (i - slice_i0)] holds the bf16-rounded value as f32.
-template <int MT>
-__device__ bool consume_gateup(Consumer& cs, const GateUpGeom& g, int g0, int n_groups,
-                               const float* s, const float* rinv, __nv_bfloat16* a, int m0,
-                               int mt, float* xch, float* slice = nullptr, int slice_i0 = 0,
-                               int slice_ld = 0) {
-  const int c = (threadIdx.x >> 5) - 1, lane = cs.lane;
-  const int pr = c & (kGroup - 1), half = c / kGroup;
-  for (int j = 0; j < n_groups; ++j) {
-    uint64_t ag[2][MT], au[2][MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) ag[0][m] = ag[1][m] = au[0][m] = au[1][m] = 0ull;
-    bool ok = true;
-    for (int ch = 0; ch < g.nchunks && ok; ++ch) {
-      const uint8_t* buf = cs.wait_full();
-      if (!buf) {
-        ok = false;
-        break;
-      }
-      const int k0 = ch * g.kc;
-      const int nv = min(g.kc, g.d - k0) / 8;
-      const uint8_t* bg = buf + (size_t)pr * g.kc * 2;
-      const uint8_t* bu = buf + (size_t)(kGroup + pr) * g.kc * 2;
-      const int kv0 = k0 / 8;
-      for (int v = lane + 32 * half; v < nv; v += 128) {  // vectors v and v + 64
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int vv = v + 64 * h;
-          if (h == 0 || vv < nv) {
-            const uint4 wg = lds128(bg + 16 * vv);
-            const uint4 wu = lds128(bu + 16 * vv);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              const float4* sp = reinterpret_cast<const float4*>(s + (int64_t)m * g.d) + kv0 + vv;
-              const float4 s0 = sp[0], s1 = sp[g.d / 8];
-              ag[h][m] = dot8(wg, s0, s1, ag[h][m]);
-              au[h][m] = dot8(wu, s0, s1, au[h][m]);
-            }
-          }
-        }
-      }
-      cs.release();
-    }
-    float gs[MT], us[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      gs[m] = warp_sum(hsum2(ag[0][m]) + hsum2(ag[1][m]));
-      us[m] = warp_sum(hsum2(au[0][m]) + hsum2(au[1][m]));
-    }
-    float* x2 = xch + ((j & 1) * kGroup + pr) * 2 * MT;
-    if (half == 1 && lane == 0) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        x2[m] = gs[m];
-        x2[MT + m] = us[m];
-      }
-    }
-    if (group_barrier_any(!ok)) return false;
-    if (half == 0) {
-      const int item = (g0 + j) * kGroup + pr;
-#pragma unroll
-      for (int m = 0; m < MT; ++m)
-        if (lane == m) {
-          const float gt = gs[m] + x2[m], ut = us[m] + x2[MT + m];
-          const __nv_bfloat16 av = __float2bfloat16_rn(silu_mul(gt * rinv[m], ut * rinv[m]));
-          if (slice)
-            slice[m * slice_ld + (item - slice_i0)] = m < mt ? __bfloat162float(av) : 0.f;
-          else if (m < mt)
-            a[(int64_t)(m0 + m) * g.I + item] = av;
-        }
-    }
-  }
-  return true;
-}
-
-// fused_decode's gate-up consumer: as consume_gateup, but each warp leaves
-// its warp-reduced gate and up sums of every group in `part` (shared memory,
-// [group][pair][half][gate, up][MT]) instead of combining the column halves
-// group by group, so that the warps meet at no barrier during the phase and
-// can run up to a ring's depth apart.  finish_slice combines them.
+// Gate-up consumer warps: pair w & 3 of every group, column half w >> 2, dot
+// each stage against x * gamma (s: two planes of float4 per token row, see
+// stage_x_gamma).  Each warp leaves its warp-reduced gate and up sums of every
+// group in `part` (shared memory, [group][pair][half][gate, up][MT]) instead
+// of combining the column halves group by group, so that the warps meet at no
+// barrier during the phase and can run up to a ring's depth apart (the
+// consumers process a stage only slightly faster than HBM delivers one, so a
+// barrier per group cost bandwidth).  finish_slice (fused_decode) or
+// finish_a_global (gateup_stream) combines them.
 template <int MT>
 __device__ bool consume_gateup_parts(Consumer& cs, const GateUpGeom& g, int n_groups,
                                      const float* s, float* part) {
@@ -501,6 +417,29 @@ __device__ void finish_slice(const float* part, int n_groups, const float* rinv,
   }
 }
 
+// gateup_stream: a[m0 + m, 4 g0 + i] = bf16(SiLU(r g) * r u) for the CTA's
+// 4 * n_groups pairs from the halves' sums in `part` (one coalesced pass).
+template <int MT>
+__device__ void finish_a_global(const float* part, int n_groups, const float* rinv, int mt,
+                                __nv_bfloat16* a, int64_t I, int m0, int g0) {
+  const int ct = threadIdx.x - 32;
+  for (int i = ct; i < n_groups * kGroup; i += kConsumers * 32) {
+    const float* q = part + i * 4 * MT;  // [half 0: g, u][half 1: g, u]
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m >= mt) continue;
+      const float gt = q[m] + q[2 * MT + m], ut = q[MT + m] + q[3 * MT + m];
+      a[(int64_t)(m0 + m) * I + (int64_t)g0 * kGroup + i] =
+          __float2bfloat16_rn(silu_mul(gt * rinv[m], ut * rinv[m]));
+    }
+  }
+}
+
+// Bytes of the halves' sums that gateup_stream keeps per CTA (consume_gateup_parts).
+__host__ __device__ constexpr size_t gateup_part_bytes(int max_groups, int mt) {
+  return align128((size_t)max_groups * kGroup * 4 * mt * sizeof(float));
+}
+
 // ---------------------------------------------------------------------------
 // Down phase.  A group is 4 consecutive W_down rows (one contiguous run);
 // a [MT x I] (bf16) sits in shared memory.  Stage layout: rows 0-3, kc bf16 per row.
@@ -549,24 +488,22 @@ __device__ void stage_a(const __nv_bfloat16* a, int I, int m0, int mt, uint8_t* 
   named_barrier_sync(kBarStage, kConsumers * 32);
 }
 
-// Consumer warps: row w & 3 of every group, column half w >> 2.
+// Consumer warps: row w & 3 of every group, column half w >> 2.  Each warp
+// leaves its warp-reduced sums in `part` ([group][row][half][MT], shared
+// memory); finish_down_out combines the halves after the phase, so the warps
+// meet at no barrier per group.
 template <int MT>
-__device__ bool consume_down(Consumer& cs, const DownGeom& g, int g0, int n_groups,
-                             const uint8_t* act, const __nv_bfloat16* residual, float* out,
-                             int m0, int mt, float* xch) {
+__device__ bool consume_down_parts(Consumer& cs, const DownGeom& g, int n_groups,
+                                   const uint8_t* act, float* part) {
   const int c = (threadIdx.x >> 5) - 1, lane = cs.lane;
   const int row = c & (kGroup - 1), half = c / kGroup;
   for (int j = 0; j < n_groups; ++j) {
     uint64_t acc[2][MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[0][m] = acc[1][m] = 0ull;
-    bool ok = true;
-    for (int ch = 0; ch < g.nchunks && ok; ++ch) {
+    for (int ch = 0; ch < g.nchunks; ++ch) {
       const uint8_t* buf = cs.wait_full();
-      if (!buf) {
-        ok = false;
-        break;
-      }
+      if (!buf) return false;
       const int k0 = ch * g.kc;
       const int nv = min(g.kc, g.I - k0) / 8;
       const uint8_t* bw = buf + (size_t)row * g.kc * 2;
@@ -585,28 +522,38 @@ __device__ bool consume_down(Consumer& cs, const DownGeom& g, int g0, int n_grou
       }
       cs.release();
     }
-    float t[MT];
+    float* dst = part + ((j * kGroup + row) * 2 + half) * MT;
 #pragma unroll
-    for (int m = 0; m < MT; ++m) t[m] = warp_sum(hsum2(acc[0][m]) + hsum2(acc[1][m]));
-    float* x2 = xch + ((j & 1) * kGroup + row) * 2 * MT;
-    if (half == 1 && lane == 0) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) x2[m] = t[m];
-    }
-    if (group_barrier_any(!ok)) return false;
-    if (half == 0) {
-      const int n = (g0 + j) * kDownRows + row;
-#pragma unroll
-      for (int m = 0; m < MT; ++m)
-        if (lane == m && m < mt) {
-          float o = t[m] + x2[m];
-          if (residual) o += __bfloat162float(residual[(int64_t)(m0 + m) * g.d + n]);
-          out[(int64_t)(m0 + m) * g.d + n] = o;
-        }
+    for (int m = 0; m < MT; ++m) {
+      const float t = warp_sum(hsum2(acc[0][m]) + hsum2(acc[1][m]));
+      if (lane == 0) dst[m] = t;
     }
   }
   return true;
 }
+
+// out[m0 + m, 4 g0 + i] = the halves' sums (+ residual), one coalesced pass.
+template <int MT>
+__device__ void finish_down_out(const float* part, int n_groups, const __nv_bfloat16* residual,
+                                float* out, int64_t d, int m0, int mt, int g0) {
+  const int ct = threadIdx.x - 32;
+  for (int i = ct; i < n_groups * kDownRows; i += kConsumers * 32) {
+    const float* q = part + i * 2 * MT;  // [half 0][half 1]
+    const int64_t n = (int64_t)g0 * kDownRows + i;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m >= mt) continue;
+      float o = q[m] + q[MT + m];
+      if (residual) o += __bfloat162float(residual[(int64_t)(m0 + m) * d + n]);
+      out[(int64_t)(m0 + m) * d + n] = o;
+    }
+  }
+}
+
+__host__ __device__ constexpr size_t down_part_bytes(int max_groups, int mt) {
+  return align128((size_t)max_groups * kDownRows * 2 * mt * sizeof(float));
+}
+
 
 // ---------------------------------------------------------------------------
 // Kernels
@@ -625,17 +572,21 @@ struct StreamParams {
   int stages, stage_bytes;
 };
 
+// act_main: bytes of the activations at the start of the dynamic shared
+// memory (x * gamma in f32, or a in bf16); the halves' sums follow them, and
+// the ring starts at act_bytes.
 template <int MT, bool GATE, bool DOWN>
-__device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_bytes) {
+__device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_main,
+                                            size_t act_bytes) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ float red[kConsumers][MT];
-  __shared__ float xch[2 * kGroup * 2 * MT];
   __shared__ CtaState st;
 
   Ring ring;
   ring.full = reinterpret_cast<uint64_t*>(smem);
   ring.empty = ring.full + kMaxStages;
   uint8_t* act = smem + kHeader;
+  float* part = reinterpret_cast<float*>(act + act_main);
   ring.stage0 = smem + kHeader + act_bytes;
   ring.stages = p.stages;
   ring.stage_bytes = p.stage_bytes;
@@ -665,17 +616,22 @@ __device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_by
     if (GATE) stage_gamma(p.gamma, p.gu.d, reinterpret_cast<float*>(act));
     grid_dependency_wait();  // inputs may be written by the previous kernel
     Consumer cs{ring, &st, p.ctl, 0, lane};
-    bool ok = true;
+    // every warp's sums of every group go to `part`; after one barrier (which
+    // also agrees on failure) the halves are combined and written out
     if (GATE) {
       float rinv[MT];
       stage_x_gamma<MT>(p.x, nullptr, p.eps, p.gu.d, m0, mt, reinterpret_cast<float*>(act),
                         red, rinv);
-      ok = consume_gateup<MT>(cs, p.gu, ga0, nga, reinterpret_cast<const float*>(act), rinv,
-                              p.a, m0, mt, xch);
+      const bool ok = consume_gateup_parts<MT>(cs, p.gu, nga, reinterpret_cast<const float*>(act),
+                                               part);
+      if (!consumer_barrier_any(kBarStage, !ok))
+        finish_a_global<MT>(part, nga, rinv, mt, p.a, p.gu.I, m0, ga0);
     }
-    if (DOWN && ok) {
+    if (DOWN) {
       stage_a<MT>(p.a, p.dn.I, m0, mt, act);
-      consume_down<MT>(cs, p.dn, gd0, ngd, act, p.residual, p.out, m0, mt, xch);
+      const bool ok = consume_down_parts<MT>(cs, p.dn, ngd, act, part);
+      if (!consumer_barrier_any(kBarStage, !ok))
+        finish_down_out<MT>(part, ngd, p.residual, p.out, p.dn.d, m0, mt, gd0);
     }
   }
   __syncthreads();
@@ -684,12 +640,16 @@ __device__ __forceinline__ void stream_body(const StreamParams& p, size_t act_by
 
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1) gateup_stream(const StreamParams p) {
-  stream_body<MT, true, false>(p, align128((size_t)MT * p.gu.d * sizeof(float)));
+  const size_t act_main = align128((size_t)MT * p.gu.d * sizeof(float));
+  const int max_groups = (p.gu.I / kGroup + gridDim.x - 1) / gridDim.x;
+  stream_body<MT, true, false>(p, act_main, act_main + gateup_part_bytes(max_groups, MT));
 }
 
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1) down_stream(const StreamParams p) {
-  stream_body<MT, false, true>(p, align128((size_t)MT * p.dn.I * 2));
+  const size_t act_main = align128((size_t)MT * p.dn.I * 2);
+  const int max_groups = (p.dn.d / kDownRows + gridDim.x - 1) / gridDim.x;
+  stream_body<MT, false, true>(p, act_main, act_main + down_part_bytes(max_groups, MT));
 }
 
 // ---------------------------------------------------------------------------
@@ -1012,9 +972,16 @@ Plan make_plan(int64_t M, int64_t d, int64_t I, bool gate, bool down, const Devi
   const size_t budget = (size_t)dev.max_smem_optin - 1024;  // static smem + slack
   for (int min_stages = 3; min_stages >= 2; --min_stages)
     for (int mt = (int)std::min<int64_t>(M, 4); mt >= 1; --mt) {
+      // activations plus the halves' sums of the CTA's groups (grid as launched)
+      const int grid_g = (int)std::min<int64_t>(I / kGroup, dev.sm_count);
+      const int grid_d = (int)std::min<int64_t>(d / kDownRows, dev.sm_count);
       size_t act = 0;
-      if (gate) act = std::max(act, align128((size_t)mt * d * sizeof(float)));
-      if (down) act = std::max(act, align128((size_t)mt * I * 2));
+      if (gate)
+        act = std::max(act, align128((size_t)mt * d * sizeof(float)) +
+                                gateup_part_bytes((int)((I / kGroup + grid_g - 1) / grid_g), mt));
+      if (down)
+        act = std::max(act, align128((size_t)mt * I * 2) +
+                                down_part_bytes((int)((d / kDownRows + grid_d - 1) / grid_d), mt));
       const size_t fixed = kHeader + act;
       if (fixed >= budget) continue;
       for (int64_t target = kMaxStageBytes; target >= 4096; target /= 2) {
