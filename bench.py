@@ -381,9 +381,10 @@ def run_ours(args) -> None:
     ms_step = elapsed_ms / args.steps
     tok_per_s_layer = M * L * args.steps * world / (elapsed_ms / 1e3)
 
-    # per-launch durations, each launch bracketed by events on the launching
-    # stream: (1) fmlp_forward, one fused kernel per layer at these token
-    # counts; (2) the same step through the two stage calls
+    # per-call durations, each call bracketed by events on the launching
+    # stream: (1) fmlp_forward (one fused kernel per layer for a single token
+    # row, three tensor-core launches for batches); (2) the same step through
+    # the two stage calls
     kernel_steps = max(1, min(args.steps, 50))
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
     fw_ms = []

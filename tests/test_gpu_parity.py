@@ -360,7 +360,7 @@ def test_bounded_wait_timeout_reports_and_recovers(fm):
     word, lets its in-flight copies land and returns; the context stays usable
     and the next call, with injection off, is correct."""
     dev = torch.device("cuda:0")
-    for M in (2, 7):   # the fused kernel, and the two-kernel path
+    for M in (2, 7):   # the fused kernel, and the tensor-core path
         p = wl.make_problem(M, 1024, 2048, seed=12)
         g = {k: v.to(dev) for k, v in p.items()}
         d, I, T = 1024, 2048, 16
