@@ -424,6 +424,31 @@ def test_fused_decode_with_shorter_down_stages(fm):
                                                                intermediate="bf16"))
 
 
+@pytest.mark.parametrize("M,d,I,launches", [(2, 4096, 14336, 3), (3, 4096, 14336, 3),
+                                            (4, 3072, 8192, 3), (2, 3072, 8192, 1),
+                                            (3, 3072, 8192, 1)])
+def test_small_batches_take_the_faster_path(fm, M, d, I, launches):
+    """2-4 token rows: the tensor-core path (three launches) on layers above
+    200 MB of weights and at 4 rows, the one-launch fused kernel otherwise;
+    both within the parity bar."""
+    p = wl.make_problem(M, d, I, sigma=0.02, seed=40 + M, residual=True)
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in p.items()}
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(g["W_gate"], g["W_up"], 16, packed)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    out = torch.full((M, d), float("nan"), dtype=torch.float32, device=dev)
+    n0 = fm.fmlp_kernel_launch_count()
+    fm.fmlp_forward(g["x"], g["gamma"], EPS, packed, 16, g["W_down"], out, ws,
+                    residual=g["residual"])
+    assert fm.fmlp_kernel_launch_count() - n0 == launches
+    torch.cuda.synchronize()
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+    got = out.cpu().double().numpy()
+    assert_parity(got, oracle_out(p, residual=True), oracle_out(p, residual=True,
+                                                               intermediate="bf16"))
+
+
 @pytest.mark.parametrize("M,d,I", [(1, 32768, 64), (4, 32768, 64), (1, 64, 65536), (3, 64, 65536),
                                    (2, 8, 8)])
 def test_maximum_and_minimum_sizes(fm, M, d, I):
