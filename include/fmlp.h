@@ -113,10 +113,11 @@ FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
  *
  * Kernels: one row (M = 1), and 2-3 rows of a layer whose weights (6 d I
  * bytes) are at most 200 MB, run one fused launch (CUDA-core dot products
- * over a TMA-streamed weight ring).  Larger batches run three launches on the
+ * over a TMA-streamed weight ring).  Other batches run three launches on the
  * tensor cores (prologue, gate-up GEMM with the SiLU*up epilogue, down GEMM)
- * when d and I are multiples of 64 and tile_T is 8 or 16; other shapes run
- * two CUDA-core streaming launches.
+ * when d and I are multiples of 64 and tile_T is 8 or 16.  Failing that, up
+ * to 4 rows run the fused launch where its shared memory allows, and the
+ * rest two CUDA-core streaming launches.
  *
  * Ordering: the kernels use programmatic dependent launch.  A kernel of this
  * library may start streaming packed_Wgu, W_down and gamma while the
