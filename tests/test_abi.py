@@ -60,6 +60,18 @@ def test_workspace_bytes():
         assert L.fmlp_workspace_bytes(M, 4096, 14336) % 256 == 0
 
 
+def test_workspace_covers_the_tensor_core_path_from_two_rows():
+    """2-4 rows may run on the tensor cores (large layers, or 4 rows): their
+    workspace must hold that path's operand copy and stream-K partials, which
+    a single row (always the fused kernel) does not need."""
+    L = fm.lib
+    tc_shape = L.fmlp_workspace_bytes(2, 4096, 14336)
+    no_tc_shape = L.fmlp_workspace_bytes(2, 4096, 14344)  # I % 64 != 0: no tensor-core path
+    assert tc_shape > no_tc_shape + (1 << 20)
+    assert L.fmlp_workspace_bytes(4, 3072, 8192) > (1 << 20)
+    assert L.fmlp_workspace_bytes(1, 4096, 14336) < (1 << 20)
+
+
 # Fake, 16-byte aligned addresses: every call below fails validation and returns
 # before touching the device, so nothing is dereferenced.
 A = 0x10000
