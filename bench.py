@@ -200,27 +200,37 @@ def layer_bits(w: wl.Workload, seed: int, layer: int) -> dict:
     return {k: wl.bf16_bits(v) for k, v in {**act, **wts}.items()}
 
 
-def oracle_call(w: wl.Workload, b: dict, ic: int):
+def oracle_call(w: wl.Workload, b: dict, ic: int, keep: bool = False):
     """One oracle evaluation of the MLP block on an I-slice of `ic` columns.
 
     Gate/up/down columns are independent terms of Eq(1), so a slice of the
     intermediate dimension is a proportional share of the layer's work.
-    Returns (algorithmic bytes, seconds).
+    Returns (algorithmic bytes, seconds), and the output if `keep`.
     """
     import oracle
     wg, wu = b["W_gate"][:ic], b["W_up"][:ic]
     wd = np.ascontiguousarray(b["W_down"][:, :ic])
     t0 = time.perf_counter()
-    oracle.fused_mlp_bf16(b["x"], b["gamma"], EPS, wg, wu, wd)
-    return algorithmic_bytes(w.M, w.d, ic), time.perf_counter() - t0
+    out = oracle.fused_mlp_bf16(b["x"], b["gamma"], EPS, wg, wu, wd)
+    dt = time.perf_counter() - t0
+    if keep:
+        return algorithmic_bytes(w.M, w.d, ic), dt, out
+    return algorithmic_bytes(w.M, w.d, ic), dt
 
 
 def oracle_sample(w: wl.Workload, seconds: float, seed: int = 0):
-    """The oracle on whole layers of the workload for about `seconds` of CPU time."""
-    done, t_total, calls = 0, 0.0, 0
+    """The oracle on whole layers of the workload for about `seconds` of CPU time.
+
+    Returns (GB/s, description, the oracle's output of layer 0): layer 0 has
+    the same inputs as the benchmark's first layer, so its output checks the
+    timed kernels' result."""
+    done, t_total, calls, ref0 = 0, 0.0, 0, None
     while True:
         b = layer_bits(w, seed, calls % w.layers)
-        nb, dt = oracle_call(w, b, w.I)
+        if calls == 0:
+            nb, dt, ref0 = oracle_call(w, b, w.I, keep=True)
+        else:
+            nb, dt = oracle_call(w, b, w.I)
         done += nb
         t_total += dt
         calls += 1
@@ -228,7 +238,7 @@ def oracle_sample(w: wl.Workload, seconds: float, seed: int = 0):
             break
     desc = (f"{calls} whole layer(s) of {w.name} (M={w.M}, d={w.d}, I={w.I}) through the fp64 "
             f"oracle (bf16 decode + numpy), {t_total:.1f} s")
-    return done / t_total / 1e9, desc
+    return done / t_total / 1e9, desc, ref0
 
 
 def run_reference(args) -> None:
@@ -493,11 +503,19 @@ def run_ours(args) -> None:
     traffic = recorded_traffic("fused_decode" if fused else "tc_gemm", w.name)
 
     if rank == 0:
-        cpu = None
+        cpu, check = None, None
         if world == 1 and not args.no_cpu_baseline:
-            v, desc = oracle_sample(w, args.cpu_seconds, seed=seed0)
+            v, desc, ref0 = oracle_sample(w, args.cpu_seconds, seed=seed0)
             cpu = {"value": round(v, 4), "unit": "GB/s", "cores": blas_threads(),
                    "kind": "oracle", "sample": desc}
+            # the timed kernels' output of layer 0 (last written by the
+            # end-to-end pass, same inputs) against the oracle
+            got0 = outs[0].cpu().double().numpy()
+            norm = float(np.linalg.norm(got0 - ref0) / max(np.linalg.norm(ref0), 1e-300))
+            elem = float(np.max(np.abs(got0 - ref0)) / max(np.max(np.abs(ref0)), 1e-300))
+            check = {"layer": 0, "rows": M, "normwise": float(f"{norm:.3e}"),
+                     "per_element": float(f"{elem:.3e}"),
+                     "within_bar": bool(norm <= 2e-3 and elem <= 1e-2)}
         line = {
             "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -521,6 +539,7 @@ def run_ours(args) -> None:
                 "fmlp_down_proj_GBps": round((2 * d * I + 2 * M * I + 4 * M * d) /
                                              (dn_avg / 1e3) / 1e9, 2)},
             "cpu_baseline": cpu,
+            "check_vs_oracle": check,
             "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                     "d2h_bytes_per_step": outs_host[0].numel() * outs_host[0].element_size(),
