@@ -107,7 +107,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
@@ -179,6 +179,14 @@ def job_gbs(bytes_per_step_per_rank: int, steps: int, world: int, elapsed_ms: fl
     """Whole-job throughput: the bytes every replica streamed over the slowest
     rank's device time (replicas do equal work, so weak scaling)."""
     return bytes_per_step_per_rank * steps * world / (elapsed_ms / 1e3) / 1e9
+
+
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
 
 
 def blas_threads() -> int:
@@ -271,6 +279,7 @@ def run_reference(args) -> None:
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, args),
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                         "host_cores": host_cores(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -291,6 +300,306 @@ def config_of(w: wl.Workload, args) -> dict:
 # the CUDA path
 # ----------------------------------------------------------------------------
 
+def check_rows(M: int) -> list:
+    """Token rows compared with the oracle inside the benchmark: all of them up
+    to 128, else 64 spread over every token tile plus the last row (the
+    parity tests compare every row)."""
+    if M <= 128:
+        return list(range(M))
+    return sorted(set(range(0, M, max(1, M // 64))) | {M - 1})
+
+
+class WorkloadRun:
+    """One workload resident on the GPU: every layer's packed gate/up and
+    W_down (+ gamma), the token rows x, one output slice per layer and a
+    workspace; step() runs the whole hot path once through the C ABI."""
+
+    def __init__(self, fm, w: wl.Workload, dev, seed0: int, layers: int = 0):
+        self.fm, self.w, self.dev = fm, w, dev
+        self.M, self.d, self.I = w.M, w.d, w.I
+        self.L = layers or w.layers
+        self.seed0 = seed0
+        self.act = wl.make_activations(w.M, w.d, seed=seed0)
+        self.x = self.act["x"].to(dev)
+        self.outs = torch.empty(self.L, w.M, w.d, dtype=torch.float32, device=dev)
+        self.layers = []
+        for l in range(self.L):
+            wts = wl.make_weights(w.d, w.I, w.sigma, seed=seed0 + l)
+            gamma = wl.normal_bf16(seed0 + l, wl.TID_GAMMA, (w.d,), mean=1.0, std=0.1).to(dev)
+            wg, wu = wts["W_gate"].to(dev), wts["W_up"].to(dev)
+            packed = torch.empty(2 * w.I, w.d, dtype=torch.bfloat16, device=dev)
+            fm.fmlp_pack(wg, wu, TILE_T, packed)
+            torch.cuda.synchronize()
+            del wg, wu
+            self.layers.append({"packed": packed, "W_down": wts["W_down"].to(dev),
+                                "gamma": gamma, "out": self.outs[l]})
+        self.ws = torch.zeros(fm.fmlp_workspace_bytes(w.M, w.d, w.I), dtype=torch.uint8,
+                              device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.graph = None
+        self.per_step = None
+
+    def step(self, x=None, outs=None, stream=None):
+        fm = self.fm
+        x = self.x if x is None else x
+        for li, ly in enumerate(self.layers):
+            out = ly["out"] if outs is None else outs[li]
+            fm.fmlp_forward(x, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], out,
+                            self.ws, stream=stream)
+
+    def capture(self, warmup: int, use_graph: bool = True) -> None:
+        """Warm-up from the host (also the library's one-time set-up, before
+        any capture), then a CUDA graph of one step."""
+        fm = self.fm
+        for _ in range(max(1, warmup)):
+            self.step()
+        torch.cuda.synchronize()
+        if not use_graph:
+            return
+        try:
+            self.graph = torch.cuda.CUDAGraph()
+            c0 = fm.fmlp_kernel_launch_count()
+            with torch.cuda.graph(self.graph):
+                self.step()
+            self.per_step = fm.fmlp_kernel_launch_count() - c0
+            torch.cuda.synchronize()
+            for _ in range(warmup):
+                self.graph.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # noqa: BLE001 -- report and launch from the host instead
+            print(f"bench: CUDA graph capture failed ({e}); launching from the host",
+                  file=sys.stderr)
+            self.graph = None
+            torch.cuda.synchronize()
+
+    def run_steps(self, n: int) -> None:
+        for _ in range(n):
+            if self.graph is not None:
+                self.graph.replay()
+            else:
+                self.step()
+
+    def timed(self, steps: int, barrier, max_over_ranks) -> tuple:
+        """Device time of exactly `steps` steps between CUDA events on the
+        launching stream, with a barrier and a synchronize on both sides, max
+        over ranks; clocks sampled during it.  Returns (ms, launches, clocks)."""
+        fm = self.fm
+        sampler = ClockSampler(self.dev.index)
+        launches0 = fm.fmlp_kernel_launch_count()
+        with sampler:
+            barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            self.run_steps(steps)
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+            barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1))
+        launches = fm.fmlp_kernel_launch_count() - launches0
+        if self.graph is not None:
+            launches = self.per_step * steps   # each replay launches the captured kernels
+        return ms, launches, sampler.summary()
+
+    def step_estimate_ms(self) -> float:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        self.run_steps(3)
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 3
+
+    def isolated_calls(self, steps: int, max_over_ranks) -> dict:
+        """Per-call durations, each call bracketed by events on the launching
+        stream: fmlp_forward, then the same step through the two stage calls."""
+        fm, stream, L = self.fm, self.stream, self.L
+        a_buf = torch.empty(self.M, self.I, dtype=torch.bfloat16, device=self.dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
+        fw_ms = []
+        for _ in range(steps):
+            for ly, (a0, a1) in zip(self.layers, ev):
+                a0.record(stream)
+                fm.fmlp_forward(self.x, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"],
+                                ly["out"], self.ws, stream=stream)
+                a1.record(stream)
+            torch.cuda.synchronize()
+            fw_ms.extend(a0.elapsed_time(a1) for a0, a1 in ev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)]
+        gu_ms, dn_ms = [], []
+        for _ in range(steps):
+            for ly, (a0, a1, a2) in zip(self.layers, ev):
+                a0.record(stream)
+                fm.fmlp_gate_up_swiglu(self.x, ly["gamma"], EPS, ly["packed"], TILE_T, a_buf,
+                                       self.ws, stream=stream)
+                a1.record(stream)
+                fm.fmlp_down_proj(a_buf, ly["W_down"], ly["out"], self.ws, stream=stream)
+                a2.record(stream)
+            torch.cuda.synchronize()
+            for a0, a1, a2 in ev:
+                gu_ms.append(a0.elapsed_time(a1))
+                dn_ms.append(a1.elapsed_time(a2))
+        return {"fmlp_forward_ms": max_over_ranks(statistics.mean(fw_ms)),
+                "fmlp_gate_up_swiglu_ms": max_over_ranks(statistics.mean(gu_ms)),
+                "fmlp_down_proj_ms": max_over_ranks(statistics.mean(dn_ms))}
+
+    def e2e(self, steps: int, barrier, max_over_ranks) -> tuple:
+        """The same step end to end, the way a serving loop runs it: every step
+        copies its input from pinned host memory and its outputs (every layer's
+        out) back to pinned host memory, both on copy streams and
+        double-buffered, so that step i's copies overlap the layers of its
+        neighbours.  The timed region starts before the first input copy and
+        ends after the last output copy.  Returns (ms, h2d bytes, d2h bytes)."""
+        dev, stream, L, M, d = self.dev, self.stream, self.L, self.M, self.d
+        x_host = self.act["x"].pin_memory()
+        outs_host = [torch.empty(L, M, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+        x_dev = [torch.empty_like(self.x) for _ in range(2)]
+        outs_dev = [self.outs, torch.empty_like(self.outs)]
+        copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_step(i):
+            b = i & 1
+            copy_in.wait_event(ev_done[b])       # step i - 2 has read x_dev[b]
+            with torch.cuda.stream(copy_in):
+                x_dev[b].copy_(x_host, non_blocking=True)
+            ev_in[b].record(copy_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])         # step i - 2's outputs have left outs_dev[b]
+            self.step(x=x_dev[b], outs=outs_dev[b], stream=stream)
+            ev_done[b].record(stream)
+            copy_out.wait_event(ev_done[b])
+            with torch.cuda.stream(copy_out):
+                outs_host[b].copy_(outs_dev[b], non_blocking=True)
+            ev_out[b].record(copy_out)
+
+        e2e_step(0)
+        e2e_step(1)
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        copy_in.wait_stream(stream)
+        for i in range(steps):
+            e2e_step(i)
+        stream.wait_event(ev_out[0])
+        stream.wait_event(ev_out[1])
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        # the last pass wrote layer 0's output of buffer 0 last when steps is even
+        self.outs_last = outs_dev[(steps - 1) & 1]
+        return (max_over_ranks(f0.elapsed_time(f1)), x_host.numel() * x_host.element_size(),
+                outs_host[0].numel() * outs_host[0].element_size())
+
+    def release(self) -> None:
+        self.graph = None
+        self.layers = []
+        self.outs = self.outs_last = None
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def peaks_of() -> tuple:
+    peaks = measured_peaks()
+    if "hbm_gbs" in peaks:
+        hbm = (float(peaks["hbm_gbs"]), "measured")
+    else:
+        hbm = (FALLBACK_HBM_GBS, "fallback")
+    if "bf16_tflops" in peaks:
+        tc = (float(peaks["bf16_tflops"]), "measured")
+    else:
+        tc = (FALLBACK_BF16_TFLOPS, "fallback")
+    return hbm, tc
+
+
+def roofline_entry(run: WorkloadRun, ms_step: float, gu_ms) -> dict:
+    """The dominant kernel against its roofline.  One kernel per layer (the
+    single-launch paths): its average launch duration is the timed region over
+    the launches in it.  Otherwise the gate-up call, timed with events around
+    each isolated call (it includes the small prologue kernel)."""
+    M, d, I, L, w = run.M, run.d, run.I, run.L, run.w
+    (peak, peak_src), (tpeak, tpeak_src) = peaks_of()
+    single = run.per_step is not None and run.per_step == L
+    if single:
+        kname = "fused_decode" if M <= 4 else "tc_layer"
+        kms = ms_step / L
+        timing = "timed region / launches (the step's only kernel, back to back in a CUDA graph)"
+        kbytes, kflops = algorithmic_bytes(M, d, I), 6 * M * d * I
+    else:
+        kname, kms = "gate-up (fmlp_gate_up_swiglu)", gu_ms
+        timing = "isolated: events around each call"
+        kbytes, kflops = gateup_bytes(M, d, I), 4 * M * d * I
+    if kflops / kbytes > tpeak * 1e12 / (peak * 1e9):
+        bound, kpeak, src, unit, work = "tensor", tpeak, tpeak_src, "TFLOP/s", kflops
+    else:
+        bound, kpeak, src, unit, work = "hbm", peak, peak_src, "GB/s", kbytes
+    achieved = work / (kms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    traffic = recorded_traffic("fused_decode" if kname == "fused_decode" else
+                               ("tc_layer" if kname == "tc_layer" else "tc_gemm"), w.name)
+    return {"bound": bound, "kernel": kname, "achieved": round(achieved, 2), "peak": kpeak,
+            "peak_source": src, "unit": unit, "frac": round(achieved / kpeak, 4),
+            "traffic": traffic, "algorithmic_per_launch": work, "avg_launch_ms": round(kms, 5),
+            "launch_timing": timing}
+
+
+def oracle_check(run: WorkloadRun, got_outs) -> dict:
+    """The timed kernels' output of layer 0 (written by the last end-to-end
+    pass, same inputs) against the oracle on the rows of check_rows."""
+    w = run.w
+    rows = check_rows(w.M)
+    b = layer_bits(w, run.seed0, 0)
+    import oracle
+    ref = oracle.fused_mlp_bf16(b["x"][rows], b["gamma"], EPS, b["W_gate"], b["W_up"],
+                                b["W_down"])
+    got = got_outs[0].cpu().double().numpy()[rows]
+    norm = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    elem = float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-300))
+    return {"layer": 0, "rows": len(rows), "normwise": float(f"{norm:.3e}"),
+            "per_element": float(f"{elem:.3e}"), "within_bar": bool(norm <= 2e-3 and elem <= 1e-2)}
+
+
+def measure_sub_workload(fm, w: wl.Workload, dev, args, barrier, max_over_ranks, rank: int,
+                         world: int) -> dict:
+    """One entry of the line's `workloads` object: the workload timed for at
+    least --min-seconds of device time, its own clocks, roofline, end-to-end
+    pass and oracle check."""
+    run = WorkloadRun(fm, w, dev, seed0=1000 * rank)
+    run.capture(args.warmup, use_graph=not args.no_graph)
+    est = run.step_estimate_ms()
+    steps = max(args.steps, int(np.ceil(args.min_seconds * 1e3 / max(est, 1e-3))))
+    ms, launches, clocks = run.timed(steps, barrier, max_over_ranks)
+    ms_step = ms / steps
+    gu_ms = None
+    if not (run.per_step is not None and run.per_step == run.L):
+        gu_ms = run.isolated_calls(max(3, min(20, steps)), max_over_ranks)["fmlp_gate_up_swiglu_ms"]
+    e2e_steps = max(2, min(4000, int(np.ceil(0.5e3 / max(est, 1e-3)))))
+    e2e_ms, h2d, d2h = run.e2e(e2e_steps, barrier, max_over_ranks)
+    bytes_step = run.L * algorithmic_bytes(w.M, w.d, w.I)
+    (peak, _), (tpeak, _) = peaks_of()
+    gbs = job_gbs(bytes_step, steps, world, ms)
+    tflops = 6 * w.M * w.d * w.I * run.L * steps * world / (ms / 1e3) / 1e12
+    entry = {
+        "config": {"M": w.M, "d": w.d, "I": w.I, "layers": run.L, "tile_T": TILE_T,
+                   "weights_per_gpu_GB": round(run.L * w.weight_bytes / 1e9, 3)},
+        "value": round(gbs, 2), "unit": "GB/s", "hbm_frac": round(gbs / world / peak, 4),
+        "tflops": round(tflops, 2), "tensor_frac": round(tflops / world / tpeak, 4),
+        "tokens_per_s_per_layer": round(w.M * run.L * steps * world / (ms / 1e3), 1),
+        "ms_per_layer": round(ms_step / run.L, 5), "steps": steps, "timed_ms": round(ms, 2),
+        "roofline": roofline_entry(run, ms_step, gu_ms),
+        "e2e": {"value": round(job_gbs(bytes_step, e2e_steps, world, e2e_ms), 2), "unit": "GB/s",
+                "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches, "cuda_graph": run.graph is not None,
+        "device_status": fm.fmlp_status_string(fm.fmlp_device_status(run.ws)),
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_oracle_check:
+        entry["check_vs_oracle"] = oracle_check(run, run.outs_last)
+    run.release()
+    return entry
+
+
 def run_ours(args) -> None:
     rank, world, local = dist_env()
     if world > 1:
@@ -304,35 +613,6 @@ def run_ours(args) -> None:
     dev = torch.device("cuda", torch.cuda.current_device())
     import token_phase_swiglu_b200 as fm
 
-    w = wl.WORKLOADS[args.workload]
-    M, d, I, L = w.M, w.d, w.I, (args.layers or w.layers)
-    seed0 = 1000 * rank
-
-    # resident weights: packed gate/up and W_down per layer (+ gamma per layer);
-    # the layers' outputs are slices of one buffer, returned with one copy
-    act = wl.make_activations(M, d, seed=seed0)
-    x = act["x"].to(dev)
-    outs = torch.empty(L, M, d, dtype=torch.float32, device=dev)
-    layers = []
-    for l in range(L):
-        wts = wl.make_weights(d, I, w.sigma, seed=seed0 + l)
-        gamma = wl.normal_bf16(seed0 + l, wl.TID_GAMMA, (d,), mean=1.0, std=0.1).to(dev)
-        wg, wu = wts["W_gate"].to(dev), wts["W_up"].to(dev)
-        packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
-        fm.fmlp_pack(wg, wu, TILE_T, packed)
-        torch.cuda.synchronize()
-        del wg, wu
-        layers.append({"packed": packed, "W_down": wts["W_down"].to(dev), "gamma": gamma,
-                       "out": outs[l]})
-    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
-    a_buf = torch.empty(M, I, dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        # the current stream (the capture stream while a graph is being captured)
-        for ly in layers:
-            fm.fmlp_forward(x, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], ly["out"], ws)
-
     def barrier():
         if world > 1:
             import torch.distributed as dist
@@ -341,181 +621,48 @@ def run_ours(args) -> None:
     def max_over_ranks(v: float) -> float:
         return reduce_max(v, dev)
 
-    # warm-up (also the one-time library set-up, before any graph capture)
-    for _ in range(max(1, args.warmup)):
-        step()
-    torch.cuda.synchronize()
+    w = wl.WORKLOADS[args.workload]
+    run = WorkloadRun(fm, w, dev, seed0=1000 * rank, layers=args.layers)
+    M, d, I, L = run.M, run.d, run.I, run.L
+    run.capture(args.warmup, use_graph=not args.no_graph)
 
-    graph = None
-    per_step = None
-    if not args.no_graph:
-        try:
-            graph = torch.cuda.CUDAGraph()
-            c0 = fm.fmlp_kernel_launch_count()
-            with torch.cuda.graph(graph):
-                step()
-            per_step = fm.fmlp_kernel_launch_count() - c0   # kernels captured per step
-            torch.cuda.synchronize()
-            for _ in range(args.warmup):
-                graph.replay()
-            torch.cuda.synchronize()
-        except Exception as e:  # noqa: BLE001 -- report and launch from the host instead
-            print(f"bench: CUDA graph capture failed ({e}); launching from the host",
-                  file=sys.stderr)
-            graph = None
-            torch.cuda.synchronize()
-
-    sampler = ClockSampler(dev.index)
-    launches0 = fm.fmlp_kernel_launch_count()
-    with sampler:
-        barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            if graph is not None:
-                graph.replay()
-            else:
-                step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-    elapsed_ms = max_over_ranks(e0.elapsed_time(e1))
-    launches = fm.fmlp_kernel_launch_count() - launches0
-    if graph is not None:
-        launches = per_step * args.steps   # each replay launches the captured kernels
-    fm_status = fm.fmlp_device_status(ws)
-
+    # the headline: exactly K timed steps
+    elapsed_ms, launches, clocks = run.timed(args.steps, barrier, max_over_ranks)
+    fm_status = fm.fmlp_device_status(run.ws)
     bytes_step = L * algorithmic_bytes(M, d, I)
     gbs = job_gbs(bytes_step, args.steps, world, elapsed_ms)
     ms_step = elapsed_ms / args.steps
     tok_per_s_layer = M * L * args.steps * world / (elapsed_ms / 1e3)
 
-    # per-call durations, each call bracketed by events on the launching
-    # stream: (1) fmlp_forward (one fused kernel per layer for a single token
-    # row, three tensor-core launches for batches); (2) the same step through
-    # the two stage calls
-    kernel_steps = max(1, min(args.steps, 50))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
-    fw_ms = []
-    for _ in range(kernel_steps):
-        for ly, (a0, a1) in zip(layers, ev):
-            a0.record(stream)
-            fm.fmlp_forward(x, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], ly["out"], ws,
-                            stream=stream)
-            a1.record(stream)
-        torch.cuda.synchronize()
-        fw_ms.extend(a0.elapsed_time(a1) for a0, a1 in ev)
-    fw_avg = max_over_ranks(statistics.mean(fw_ms))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)]
-    gu_ms, dn_ms = [], []
-    for _ in range(kernel_steps):
-        for ly, (a0, a1, a2) in zip(layers, ev):
-            a0.record(stream)
-            fm.fmlp_gate_up_swiglu(x, ly["gamma"], EPS, ly["packed"], TILE_T, a_buf, ws,
-                                   stream=stream)
-            a1.record(stream)
-            fm.fmlp_down_proj(a_buf, ly["W_down"], ly["out"], ws, stream=stream)
-            a2.record(stream)
-        torch.cuda.synchronize()
-        for a0, a1, a2 in ev:
-            gu_ms.append(a0.elapsed_time(a1))
-            dn_ms.append(a1.elapsed_time(a2))
-    gu_avg = max_over_ranks(statistics.mean(gu_ms))
-    dn_avg = max_over_ranks(statistics.mean(dn_ms))
-
-    # end to end, the way a serving loop runs it: every step copies its input
-    # from pinned host memory and its outputs (every layer's out) back to
-    # pinned host memory, both on copy streams and double-buffered, so that
-    # step i's copies overlap the layers of its neighbours.  The timed region
-    # starts before the first input copy and ends after the last output copy.
-    x_host = act["x"].pin_memory()
-    outs_host = [torch.empty(L, M, d, dtype=torch.float32).pin_memory() for _ in range(2)]
-    x_dev = [torch.empty_like(x) for _ in range(2)]
-    outs_dev = [outs, torch.empty_like(outs)]
-    copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    e2e_steps = max(1, min(args.steps, 200))
-
-    def e2e_step(i):
-        b = i & 1
-        copy_in.wait_event(ev_done[b])       # step i - 2 has read x_dev[b]
-        with torch.cuda.stream(copy_in):
-            x_dev[b].copy_(x_host, non_blocking=True)
-        ev_in[b].record(copy_in)
-        stream.wait_event(ev_in[b])
-        stream.wait_event(ev_out[b])         # step i - 2's outputs have left outs_dev[b]
-        for li, ly in enumerate(layers):
-            fm.fmlp_forward(x_dev[b], ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"],
-                            outs_dev[b][li], ws, stream=stream)
-        ev_done[b].record(stream)
-        copy_out.wait_event(ev_done[b])
-        with torch.cuda.stream(copy_out):
-            outs_host[b].copy_(outs_dev[b], non_blocking=True)
-        ev_out[b].record(copy_out)
-
-    e2e_step(0)
-    e2e_step(1)
-    torch.cuda.synchronize()
-    barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    copy_in.wait_stream(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    stream.wait_event(ev_out[0])
-    stream.wait_event(ev_out[1])
-    f1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    iso = run.isolated_calls(max(1, min(args.steps, 50)), max_over_ranks)
+    e2e_steps = max(2, min(args.steps, 200))
+    e2e_ms, h2d, d2h = run.e2e(e2e_steps, barrier, max_over_ranks)
     e2e_gbs = job_gbs(bytes_step, e2e_steps, world, e2e_ms)
+    roof = roofline_entry(run, ms_step, iso["fmlp_gate_up_swiglu_ms"])
+    (peak, _), _ = peaks_of()
 
-    peaks = measured_peaks()
-    if "hbm_gbs" in peaks:
-        peak, peak_src = float(peaks["hbm_gbs"]), "measured"
-    else:
-        peak, peak_src = FALLBACK_HBM_GBS, "fallback"
-    fused = per_step is not None and per_step == L   # one kernel per layer
-    if "bf16_tflops" in peaks:
-        tpeak, tpeak_src = float(peaks["bf16_tflops"]), "measured"
-    else:
-        tpeak, tpeak_src = FALLBACK_BF16_TFLOPS, "fallback"
-    gu_flops = 4 * M * d * I                      # algorithmic gate-up FLOPs
-    timing = "isolated: events around each call"
-    if fused:
-        # the step is nothing but this kernel, once per layer: its average
-        # launch duration is the timed region over the launches in it
-        kname, kbytes = "fused_decode", algorithmic_bytes(M, d, I)
-        kms = ms_step / L
-        timing = "timed region / launches (the step's only kernel, back to back in a CUDA graph)"
-        bound, kpeak, kpeak_src, kunit, kwork = "hbm", peak, peak_src, "GB/s", kbytes
-    else:
-        kname, kbytes, kms = "gate-up (fmlp_gate_up_swiglu)", gateup_bytes(M, d, I), gu_avg
-        # tensor-bound when the gate-up's intensity exceeds the measured ridge point
-        if gu_flops / kbytes > tpeak * 1e12 / (peak * 1e9):
-            bound, kpeak, kpeak_src, kunit, kwork = "tensor", tpeak, tpeak_src, "TFLOP/s", gu_flops
-        else:
-            bound, kpeak, kpeak_src, kunit, kwork = "hbm", peak, peak_src, "GB/s", kbytes
-    k_achieved = kwork / (kms / 1e3) / (1e12 if kunit == "TFLOP/s" else 1e9)
-    traffic = recorded_traffic("fused_decode" if fused else "tc_gemm", w.name)
+    cpu, check = None, None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, _ = oracle_sample(w, args.cpu_seconds, seed=run.seed0)
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": blas_threads(),
+               "host_cores": host_cores(), "kind": "oracle", "sample": desc}
+    if rank == 0 and not args.no_oracle_check:
+        check = oracle_check(run, run.outs_last)
+    graph_used = run.graph is not None
+    run.release()
+    del run
+
+    # every other workload (and the headline's own, timed for a second), one
+    # entry each
+    subs = {}
+    names = [] if args.workloads == "none" else (
+        list(wl.WORKLOADS) if args.workloads == "all" else args.workloads.split(","))
+    for name in names:
+        subs[name] = measure_sub_workload(fm, wl.WORKLOADS[name], dev, args, barrier,
+                                          max_over_ranks, rank, world)
 
     if rank == 0:
-        cpu, check = None, None
-        if world == 1 and not args.no_cpu_baseline:
-            v, desc, ref0 = oracle_sample(w, args.cpu_seconds, seed=seed0)
-            cpu = {"value": round(v, 4), "unit": "GB/s", "cores": blas_threads(),
-                   "kind": "oracle", "sample": desc}
-            # the timed kernels' output of layer 0 (last written by the
-            # end-to-end pass, same inputs) against the oracle
-            got0 = outs[0].cpu().double().numpy()
-            norm = float(np.linalg.norm(got0 - ref0) / max(np.linalg.norm(ref0), 1e-300))
-            elem = float(np.max(np.abs(got0 - ref0)) / max(np.max(np.abs(ref0)), 1e-300))
-            check = {"layer": 0, "rows": M, "normwise": float(f"{norm:.3e}"),
-                     "per_element": float(f"{elem:.3e}"),
-                     "within_bar": bool(norm <= 2e-3 and elem <= 1e-2)}
+        gu_ms, dn_ms = iso["fmlp_gate_up_swiglu_ms"], iso["fmlp_down_proj_ms"]
         line = {
             "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -523,35 +670,29 @@ def run_ours(args) -> None:
             "data": "synthetic", "config": config_of(w, args),
             "hbm_frac": round(gbs / world / peak, 4),
             "tokens_per_s_per_layer": round(tok_per_s_layer, 1),
-            "roofline": {"bound": bound, "kernel": kname,
-                         "achieved": round(k_achieved, 2), "peak": kpeak,
-                         "peak_source": kpeak_src, "unit": kunit,
-                         "frac": round(k_achieved / kpeak, 4), "traffic": traffic,
-                         "algorithmic_per_launch": kwork, "avg_launch_ms": round(kms, 5),
-                         "launch_timing": timing},
+            "roofline": roof,
             "tflops": round(6 * M * d * I * L * args.steps * world / (elapsed_ms / 1e3) / 1e12, 2),
             "isolated_calls": {
                 "note": "each call bracketed by its own events (no overlap with its neighbours)",
-                "fmlp_forward_ms": round(fw_avg, 5),
-                "fmlp_gate_up_swiglu_ms": round(gu_avg, 5),
-                "fmlp_gate_up_swiglu_GBps": round(gateup_bytes(M, d, I) / (gu_avg / 1e3) / 1e9, 2),
-                "fmlp_down_proj_ms": round(dn_avg, 5),
+                "fmlp_forward_ms": round(iso["fmlp_forward_ms"], 5),
+                "fmlp_gate_up_swiglu_ms": round(gu_ms, 5),
+                "fmlp_gate_up_swiglu_GBps": round(gateup_bytes(M, d, I) / (gu_ms / 1e3) / 1e9, 2),
+                "fmlp_down_proj_ms": round(dn_ms, 5),
                 "fmlp_down_proj_GBps": round((2 * d * I + 2 * M * I + 4 * M * d) /
-                                             (dn_avg / 1e3) / 1e9, 2)},
+                                             (dn_ms / 1e3) / 1e9, 2)},
             "cpu_baseline": cpu,
             "check_vs_oracle": check,
             "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s",
-                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-                    "d2h_bytes_per_step": outs_host[0].numel() * outs_host[0].element_size(),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "copies": "pinned host buffers, copy streams, double-buffered across steps"},
             "gpu_launches": launches,
-            "cuda_graph": graph is not None,
+            "cuda_graph": graph_used,
             "device_status": fm.fmlp_status_string(fm_status),
-            "clocks": sampler.summary(),
+            "clocks": clocks,
+            "workloads": subs,
         }
         print(json.dumps(line), flush=True)
 
-    del graph
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -569,6 +710,12 @@ def main() -> None:
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling captures only)")
+    ap.add_argument("--workloads", default="all",
+                    help="comma list of workloads measured as entries of the line's `workloads` "
+                         "object, 'all' (default) or 'none'")
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="device time each `workloads` entry is timed for, at least")
+    ap.add_argument("--no-oracle-check", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

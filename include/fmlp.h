@@ -92,6 +92,12 @@ FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
  * fmlp_forward -- the whole MLP block (steps a1-a6): RMSNorm, interleaved
  * gate-up contraction, SiLU*up epilogue, down projection, optional residual.
  *
+ * FastTPS section 三: Eq(1), O = W_down(SiLU(W_gate h) * (W_up h)), and the
+ * MLP execution flow RMSNorm -> interleaved gate-up Matmul -> siLu_Mul ->
+ * down projection (Figure 4 parts 1-3); section 五, Fusion MLP Steps 1-3 (the
+ * block as one kernel).  The residual add is this library's own option; the
+ * pages do not name it.
+ *
  *   x          : bf16 [M x d] token rows
  *   M          : token rows, >= 0
  *   gamma      : bf16 [d] RMSNorm weight (multiplies directly)
@@ -107,8 +113,9 @@ FMLP_API size_t fmlp_workspace_bytes(int64_t M, int64_t d, int64_t I);
  * f32 precision (CUDA-core path) or as an exact hi+lo bf16 pair (tensor-core
  * path); accumulation is f32; SiLU is evaluated in f32 (on the tensor-core
  * path with the hardware exp2 and reciprocal approximations, relative error
- * about 1e-6); a is rounded once to bf16 (round to nearest even); out is f32.  out is written by several thread blocks adding into it
- * (f32 atomics), so the summation order, and the last bits of out, may differ
+ * about 1e-6); a is rounded once to bf16 (round to nearest even); out is
+ * f32.  out is written by several thread blocks adding into it (f32
+ * atomics), so the summation order, and the last bits of out, may differ
  * from run to run.  out must not overlap any input.
  *
  * Kernels: one row (M = 1), and 2-3 rows of a layer whose weights (6 d I
@@ -135,7 +142,10 @@ FMLP_API fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, f
  * fmlp_gate_up_swiglu -- steps a1-a4 alone: writes the bf16 intermediate
  *     a[m,i] = bf16( SiLU(r[m] * g[m,i]) * r[m] * u[m,i] )
  * with g, u the contractions of x*gamma with the gate and up rows of
- * packed_Wgu.  Arguments as in fmlp_forward; `a` is bf16 [M x I] and must not
+ * packed_Wgu.  FastTPS section 三, Eq(1) inside W_down(...) and Figure 4
+ * parts 1-2 (RMSNorm, interleaved gate-up Matmul, siLu_Mul); section 五,
+ * Fusion MLP Steps 1-2; the llama.cpp PR paragraph (gate and up rows
+ * alternate and the GLU is applied in the same pass).  Arguments as in fmlp_forward; `a` is bf16 [M x I] and must not
  * overlap the workspace.
  */
 FMLP_API fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* gamma, float eps,
@@ -145,6 +155,9 @@ FMLP_API fmlp_status fmlp_gate_up_swiglu(const void* x, int64_t M, const void* g
 
 /*
  * fmlp_down_proj -- steps a5-a6 alone: out = a W_down^T (+ residual).
+ * FastTPS section 三, the outer W_down(...) of Eq(1) and Figure 4 part 3
+ * (down projection); section 五, Fusion MLP Step 3 (read with Eq(1): the
+ * element-wise product is already in a).
  *   a : bf16 [M x I]; other arguments as in fmlp_forward.
  */
 FMLP_API fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t d,
@@ -171,14 +184,20 @@ FMLP_API fmlp_status fmlp_device_status(void* workspace, void* stream);
  * Instead of a caller workspace it uses one scratch buffer of
  * FMLP_NOALLOC_SCRATCH_BYTES that the library keeps in every GPU's memory
  * from the moment the library is loaded until the process exits.  The call
- * itself allocates nothing.  The first call on a device looks up the
- * buffer's address for that device (cudaGetSymbolAddress) and caches it;
- * make that first call before any stream capture.
+ * itself allocates nothing.  The first call on a device, and the first after
+ * the device's context changed (cudaDeviceReset, or another context made
+ * current), looks up the buffer's address in that context
+ * (cudaGetSymbolAddress) and caches it for that device and context; make
+ * that first call before any stream capture.
  *
  * Arguments, layouts and precision are those of fmlp_forward, minus the
  * workspace.  Requests whose workspace (fmlp_workspace_bytes(M, d, I)) would
  * exceed FMLP_NOALLOC_SCRATCH_BYTES are rejected with FMLP_ERR_UNSUPPORTED
- * before anything is enqueued.  Each call first clears the buffer's control
+ * before anything is enqueued.  Of the benchmarked shapes, the tiny layer
+ * (M=4, d=256, I=688), the Phi-3-mini decode layer (M=1, d=3072, I=8192)
+ * and the Llama-3.1-8B decode layer at M=1 and M=8 (d=4096, I=14336) fit;
+ * the 8B layer at M=32 (11.4 MiB), the 70B verify layer (M=128, 51 MiB)
+ * and the 8B prefill chunk (M=2048, 128 MiB) do not.  Each call first clears the buffer's control
  * words on `stream`, then runs the fmlp_forward kernels on it.  Every call in
  * the process shares the one buffer: calls that may overlap on the GPU (two
  * streams, or two threads) race and must not be issued.  A device-side

@@ -131,3 +131,35 @@ def test_binding_checks_dtypes():
     x = torch.zeros(2, 8, dtype=torch.float32)
     with pytest.raises(TypeError):
         fm.fmlp_pack(x, x, 8, x)
+
+
+def test_binding_checks_shapes_and_device_before_the_library():
+    """The Python wrappers reject a tensor of the wrong dtype (TypeError), shape
+    or device (ValueError) before any pointer reaches the C ABI: a short or
+    bf16 `out` would otherwise be written past its end."""
+    import torch
+    d, I, M = 16, 32, 2
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    x, gamma, packed, Wd = bf(M, d), bf(d), bf(2 * I, d), bf(d, I)
+    out = torch.zeros(M, d, dtype=torch.float32)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        fm.fmlp_forward(x, gamma, 1e-5, packed, 16, Wd, out.to(torch.bfloat16), ws)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_forward(x, gamma, 1e-5, packed, 16, Wd, out[:1], ws)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_forward(x, bf(d + 8), 1e-5, packed, 16, Wd, out, ws)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_forward(x, gamma, 1e-5, bf(I, d), 16, Wd, out, ws)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_forward(x, gamma, 1e-5, packed, 16, Wd, out, ws, residual=bf(M + 1, d))
+    with pytest.raises(ValueError, match="rows"):
+        fm.fmlp_forward(x, gamma, 1e-5, packed, 16, bf(d + 8, I), out, ws)
+    with pytest.raises(ValueError, match="CUDA"):     # host memory is not device memory
+        fm.fmlp_forward(x, gamma, 1e-5, packed, 16, Wd, out, ws)
+    with pytest.raises(ValueError, match="CUDA"):
+        fm.fmlp_forward_noalloc(x, gamma, 1e-5, packed, 16, Wd, out)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_down_proj(bf(M, I), Wd, out[:, :8], ws)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_gate_up_swiglu(x, gamma, 1e-5, packed, 16, bf(M + 1, I), ws)

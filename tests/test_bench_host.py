@@ -46,3 +46,13 @@ def test_warmup_floor():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                           "--warmup", "2"], capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0
+
+
+def test_bench_oracle_check_rows_reach_every_token_tile():
+    # all rows up to 128; else rows in every 128-row gate-up and 256-row down
+    # token tile, first and last row included
+    assert bench.check_rows(128) == list(range(128))
+    rows = bench.check_rows(2048)
+    assert rows[0] == 0 and rows[-1] == 2047 and len(rows) <= 80
+    assert {r // 128 for r in rows} == set(range(16))
+    assert {r // 256 for r in rows} == set(range(8))

@@ -72,7 +72,7 @@ class FmlpError(RuntimeError):
         super().__init__(f"{where}: {msg}")
 
 
-def _check(status: int, where: str) -> None:
+def _check_status(status: int, where: str) -> None:
     if status != FMLP_OK:
         raise FmlpError(status, where)
 
@@ -98,6 +98,69 @@ def _stream(stream):
 def _bf16(t, name):
     if t is not None and t.dtype != torch.bfloat16:
         raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+
+
+def _check(t, name, dtype, shape=None, optional=False):
+    """Check one tensor argument before its pointer goes to the library: the
+    dtype (TypeError), the exact shape and contiguity (ValueError).  Together
+    with _on_device (the library launches on the current device), nothing
+    malformed reaches the C ABI."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _on_device(**tensors):
+    """Every given tensor lives on the current CUDA device (checked after the
+    dtypes and shapes of all of them)."""
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.device.index != torch.cuda.current_device():
+            raise ValueError(f"{name} is on {t.device}, but the current device is "
+                             f"cuda:{torch.cuda.current_device()}")
+
+
+def _check_workspace(ws, need: int):
+    _check(ws, "workspace", None)
+    if ws.numel() * ws.element_size() < need:
+        raise ValueError(f"workspace holds {ws.numel() * ws.element_size()} bytes, "
+                         f"{need} needed")
+
+
+def _dims2(t, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor, got {type(t).__name__}")
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    return t.shape
+
+
+def _check_forward_args(x, gamma, packed, W_down, out, residual):
+    """Shapes of the MLP block's tensors: (M, d, I)."""
+    _bf16(x, "x")
+    M, d = _dims2(x, "x")
+    _bf16(W_down, "W_down")
+    d2, I = _dims2(W_down, "W_down")
+    if d2 != d:
+        raise ValueError(f"W_down has {d2} rows, x has {d} columns")
+    _check(x, "x", torch.bfloat16, (M, d))
+    _check(gamma, "gamma", torch.bfloat16, (d,))
+    _check(packed, "packed", torch.bfloat16, (2 * I, d))
+    _check(W_down, "W_down", torch.bfloat16, (d, I))
+    _check(residual, "residual", torch.bfloat16, (M, d), optional=True)
+    return M, d, I
 
 
 def fmlp_status_string(status: int) -> str:
@@ -129,23 +192,27 @@ def fmlp_workspace_bytes(M: int, d: int, I: int) -> int:
 def fmlp_pack(W_gate, W_up, tile_T: int, packed, stream=None) -> None:
     """packed [2I x d] <- rows of W_gate / W_up [I x d] interleaved at tile tile_T."""
     _bf16(W_gate, "W_gate"); _bf16(W_up, "W_up"); _bf16(packed, "packed")
-    I, d = W_gate.shape
-    _check(lib.fmlp_pack(_ptr(W_gate), _ptr(W_up), d, I, tile_T, _ptr(packed), _stream(stream)),
-           "fmlp_pack")
+    I, d = _dims2(W_gate, "W_gate")
+    _check(W_gate, "W_gate", torch.bfloat16, (I, d))
+    _check(W_up, "W_up", torch.bfloat16, (I, d))
+    _check(packed, "packed", torch.bfloat16, (2 * I, d))
+    _on_device(W_gate=W_gate, W_up=W_up, packed=packed)
+    _check_status(lib.fmlp_pack(_ptr(W_gate), _ptr(W_up), d, I, tile_T, _ptr(packed),
+                                _stream(stream)), "fmlp_pack")
 
 
 def fmlp_forward(x, gamma, eps: float, packed, tile_T: int, W_down, out, workspace,
                  residual=None, stream=None) -> None:
     """out [M x d] (f32) <- RMSNorm + gated MLP (+ residual) of x [M x d]."""
-    for t, n in ((x, "x"), (gamma, "gamma"), (packed, "packed"), (W_down, "W_down"),
-                 (residual, "residual")):
-        _bf16(t, n)
-    M, d = x.shape
-    I = W_down.shape[1]
-    _check(lib.fmlp_forward(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T, _ptr(W_down),
-                            d, I, _ptr(residual), _ptr(out), _ptr(workspace),
-                            workspace.numel() * workspace.element_size(), _stream(stream)),
-           "fmlp_forward")
+    M, d, I = _check_forward_args(x, gamma, packed, W_down, out, residual)
+    _check(out, "out", torch.float32, (M, d))
+    _check_workspace(workspace, fmlp_workspace_bytes(M, d, I))
+    _on_device(x=x, gamma=gamma, packed=packed, W_down=W_down, residual=residual, out=out,
+               workspace=workspace)
+    _check_status(lib.fmlp_forward(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T,
+                                   _ptr(W_down), d, I, _ptr(residual), _ptr(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+                  "fmlp_forward")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20   # FMLP_NOALLOC_SCRATCH_BYTES in include/fmlp.h
@@ -155,42 +222,53 @@ def fmlp_forward_noalloc(x, gamma, eps: float, packed, tile_T: int, W_down, out,
                          stream=None) -> None:
     """fmlp_forward without a workspace, for callers that cannot allocate device
     memory (the library's own fixed scratch buffer is used; see include/fmlp.h)."""
-    for t, n in ((x, "x"), (gamma, "gamma"), (packed, "packed"), (W_down, "W_down"),
-                 (residual, "residual")):
-        _bf16(t, n)
-    M, d = x.shape
-    I = W_down.shape[1]
-    _check(lib.fmlp_forward_noalloc(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T,
-                                    _ptr(W_down), d, I, _ptr(residual), _ptr(out),
-                                    _stream(stream)),
-           "fmlp_forward_noalloc")
+    M, d, I = _check_forward_args(x, gamma, packed, W_down, out, residual)
+    _check(out, "out", torch.float32, (M, d))
+    _on_device(x=x, gamma=gamma, packed=packed, W_down=W_down, residual=residual, out=out)
+    _check_status(lib.fmlp_forward_noalloc(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T,
+                                           _ptr(W_down), d, I, _ptr(residual), _ptr(out),
+                                           _stream(stream)),
+                  "fmlp_forward_noalloc")
 
 
 def fmlp_gate_up_swiglu(x, gamma, eps: float, packed, tile_T: int, a, workspace,
                         stream=None) -> None:
     """a [M x I] (bf16) <- SiLU(gate) * up of RMSNorm(x) against packed gate/up rows."""
-    for t, n in ((x, "x"), (gamma, "gamma"), (packed, "packed"), (a, "a")):
-        _bf16(t, n)
-    M, d = x.shape
-    I = a.shape[1]
-    _check(lib.fmlp_gate_up_swiglu(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T, d, I,
-                                   _ptr(a), _ptr(workspace),
-                                   workspace.numel() * workspace.element_size(), _stream(stream)),
-           "fmlp_gate_up_swiglu")
+    _bf16(x, "x"); _bf16(a, "a")
+    M, d = _dims2(x, "x")
+    _, I = _dims2(a, "a")
+    _check(x, "x", torch.bfloat16, (M, d))
+    _check(gamma, "gamma", torch.bfloat16, (d,))
+    _check(packed, "packed", torch.bfloat16, (2 * I, d))
+    _check(a, "a", torch.bfloat16, (M, I))
+    _check_workspace(workspace, fmlp_workspace_bytes(M, d, I))
+    _on_device(x=x, gamma=gamma, packed=packed, a=a, workspace=workspace)
+    _check_status(lib.fmlp_gate_up_swiglu(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T, d,
+                                          I, _ptr(a), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream)),
+                  "fmlp_gate_up_swiglu")
 
 
 def fmlp_down_proj(a, W_down, out, workspace, residual=None, stream=None) -> None:
     """out [M x d] (f32) <- a [M x I] W_down^T (+ residual)."""
-    for t, n in ((a, "a"), (W_down, "W_down"), (residual, "residual")):
-        _bf16(t, n)
-    M, I = a.shape
-    d = W_down.shape[0]
-    _check(lib.fmlp_down_proj(_ptr(a), M, _ptr(W_down), d, I, _ptr(residual), _ptr(out),
-                              _ptr(workspace), workspace.numel() * workspace.element_size(),
-                              _stream(stream)),
-           "fmlp_down_proj")
+    _bf16(a, "a"); _bf16(W_down, "W_down")
+    M, I = _dims2(a, "a")
+    d, _ = _dims2(W_down, "W_down")
+    _check(a, "a", torch.bfloat16, (M, I))
+    _check(W_down, "W_down", torch.bfloat16, (d, I))
+    _check(residual, "residual", torch.bfloat16, (M, d), optional=True)
+    _check(out, "out", torch.float32, (M, d))
+    _check_workspace(workspace, fmlp_workspace_bytes(M, d, I))
+    _on_device(a=a, W_down=W_down, residual=residual, out=out, workspace=workspace)
+    _check_status(lib.fmlp_down_proj(_ptr(a), M, _ptr(W_down), d, I, _ptr(residual), _ptr(out),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)),
+                  "fmlp_down_proj")
 
 
 def fmlp_device_status(workspace, stream=None) -> int:
     """Synchronise, read and clear the workspace's device status word; returns the status."""
+    _check(workspace, "workspace", None)
+    _on_device(workspace=workspace)
     return int(lib.fmlp_device_status(_ptr(workspace), _stream(stream)))

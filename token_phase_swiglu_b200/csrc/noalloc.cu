@@ -12,10 +12,16 @@
 // The buffer is a file-scope __device__ array, so every GPU that loads the
 // library reserves FMLP_NOALLOC_SCRATCH_BYTES until the process exits.  On
 // the host the array's name is only a stand-in for the symbol, not a device
-// address; the address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, and cached.
+// address; the address is looked up with cudaGetSymbolAddress, with the
+// device current, once per device and CUDA context, and cached.  The cache
+// is keyed by the context as well as the device number: after
+// cudaDeviceReset, or under a context other than the primary one, the
+// module is loaded again at a new address and the old one must not be used.
 #include "fmlp.h"
 #include "internal.h"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <mutex>
@@ -28,22 +34,60 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchEntry {
+  CUcontext ctx = nullptr;  // context the address belongs to
+  void* ptr = nullptr;
+};
+ScratchEntry g_scratch_ptr[kMaxDevices];
 
-// Device address of g_scratch on the current device (looked up on first use).
+// cuCtxGetCurrent from the driver, fetched once through the runtime (the
+// library does not link libcuda).
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+cudaError_t g_ctx_err = cudaSuccess;
+std::once_flag g_ctx_once;
+
+cudaError_t current_context(CUcontext* ctx) {
+  std::call_once(g_ctx_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    g_ctx_err = cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000,
+                                                 cudaEnableDefault, &q);
+    if (g_ctx_err == cudaSuccess && q != cudaDriverEntryPointSuccess)
+      g_ctx_err = cudaErrorNotSupported;
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  if (g_ctx_err != cudaSuccess) return g_ctx_err;
+  *ctx = nullptr;  // none current yet is not an error here
+  return g_ctx_current(ctx) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
+
+// Device address of g_scratch in the current device's current context,
+// looked up on the first call in that context and cached for it.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  CUcontext ctx = nullptr;
+  e = current_context(&ctx);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+  ScratchEntry& ent = g_scratch_ptr[dev];
+  if (ctx && ent.ctx == ctx && ent.ptr) {
+    *out = ent.ptr;
+    return cudaSuccess;
   }
-  *out = g_scratch_ptr[dev];
+  // The lookup also makes the device's primary context current when no
+  // context is, so the context is read again after it.
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_scratch);
+  if (e != cudaSuccess) return e;
+  e = current_context(&ctx);
+  if (e != cudaSuccess) return e;
+  if (!ctx) return cudaErrorDeviceUninitialized;
+  ent.ctx = ctx;
+  ent.ptr = p;
+  *out = p;
   return cudaSuccess;
 }
 
