@@ -11,8 +11,8 @@ the buffer as the first one left it), over shapes whose order sends a fused
 decode call with a wider d after calls that wrote the intermediate, and check
 each output three ways: against the fp64 oracle at the parity bar, against
 the oracle with a bf16 intermediate at the tight diagnostic bar, and against
-fmlp_forward with a caller workspace at 1e-5 (the same kernels; only the
-order of the f32 atomic adds into out differs).  One more test makes a call
+fmlp_forward with a caller workspace at 1e-4 (the same kernels; only the
+order of f32 sums differs, see TOL_SAME_KERNELS).  One more test makes a call
 time out on purpose (host-controlled fault injection: the producers withhold
 their last stage, so the bounded waits expire) and checks that the next call
 is correct, because each call clears the buffer's control words first.
@@ -28,7 +28,14 @@ import workloads as wl
 
 EPS = 1e-5
 TOL_NORM, TOL_ELEM, TIGHT_FRAC = 2e-3, 1e-2, 0.25
-TOL_SAME_KERNELS = 1e-5
+# Both entry points run the same kernels, but a gate-up tile split between
+# two thread blocks is finished by whichever arrives last, so the f32
+# summation order of its accumulators, and with it the bf16 rounding of an
+# occasional element of a, can differ from run to run.  One such element
+# moves out by about a bf16 step of a / sqrt(M I) of the output norm (2e-5 to
+# 4e-5 at these sizes); a dropped share of the contraction or a stale a costs
+# orders of magnitude more.
+TOL_SAME_KERNELS = 1e-4
 
 
 def _errors(got, ref):

@@ -3,6 +3,7 @@
 #include "fmlp.h"
 #include "internal.h"
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <mutex>
@@ -39,6 +40,36 @@ inline uint32_t* status_word(void* workspace) { return (uint32_t*)workspace; }
 bool use_tc(int64_t M, int64_t d, int64_t I, int T) {
   if (M < 2 || !tc_supported(M, d, I, T)) return false;
   return M > kFusedMaxM || M >= 4 || 6 * d * I > (int64_t)200000000;
+}
+
+LayerWorkspace layer_workspace(void* workspace, const WorkspaceLayout& L) {
+  char* w = (char*)workspace;
+  LayerWorkspace t;
+  t.b_hl = w + L.b_hl;
+  t.a = w + L.a;
+  t.rinv = (float*)(w + L.rinv);
+  t.partials = (float*)(w + L.partials);
+  t.counters = (uint32_t*)(w + L.counters);
+  t.ncounters = (int)L.ncounters;
+  t.ticket = (uint32_t*)(w + L.ticket);
+  t.inited = (uint32_t*)(w + L.inited);
+  t.done = (uint32_t*)(w + L.done);
+  t.gu_done = (uint32_t*)(w + L.gu_done);
+  t.hl_done = (uint32_t*)(w + L.hl_done);
+  t.a_ready = (uint32_t*)(w + L.a_ready);
+  t.status = status_word(workspace);
+  return t;
+}
+
+// Of the tensor-core batches, the one-launch layer kernel takes 2-8 rows of
+// a layer above 200 MB of weights, where it is the faster one; the three
+// launches the rest.  Measured on B200, four 8B-shaped layers back to back
+// (d = 4096, I = 14336; us per layer, three launches / one launch): M=2 63.1 /
+// 61.9, M=4 63.8 / 62.2, M=8 63.8 / 62.5, M=12 65.4 / 66.1, M=16 65.6 / 66.6,
+// M=32 71.0 / 72.3, M=64 84.6 / 88.6; Phi-3-shaped (151 MB) M=4 36.7 / 38.6.
+bool use_layer(int64_t M, int64_t d, int64_t I, int T, const DeviceInfo& dev) {
+  return M >= 2 && M <= 8 && 6 * d * I > (int64_t)200000000 &&
+         layer_supported(M, d, I, T, dev);
 }
 
 TcWorkspace tc_workspace(void* workspace, const WorkspaceLayout& L) {
@@ -114,21 +145,27 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
   L.inited = off + 64;
   L.done = off + 128;
   L.ticket = off + 192;
+  L.gu_done = off + 224;
+  L.hl_done = off + 240;
   off += 256;
   L.zero_end = off;
   L.a = off;
   off += align256((size_t)M * (size_t)I * 2);
-  if (M >= 2 && tc_supported(M, d, I, 16)) {  // the tensor-core path may run
+  if (M >= 2 && tc_supported(M, d, I, 16)) {  // the tensor-core paths may run
     const TcSizes z = tc_sizes(M, d, I, kTcMaxCtas);
+    const LayerSizes zl = layer_sizes(M, d, I, kTcMaxCtas);
     L.b_hl = off;
-    off += align256(z.b_hl);
+    off += align256(std::max(z.b_hl, zl.b_hl));
     L.rinv = off;
-    off += align256(z.rinv);
+    off += align256(std::max(z.rinv, zl.rinv));
     L.partials = off;
-    off += align256(z.partials);
+    off += align256(std::max(z.partials, zl.partials));
     L.counters = off;
-    L.ncounters = z.counters / 4;
-    off += align256(z.counters);
+    const size_t counters = std::max(z.counters, zl.counters);
+    L.ncounters = counters / 4;
+    off += align256(counters);
+    L.a_ready = off;
+    off += align256(zl.a_ready);
   }
   L.total = off;
   return L;
@@ -271,6 +308,9 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
     uint32_t* done = (uint32_t*)((char*)workspace + L.done);
     e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out,
                             ticket, inited, done, status, *dev, s);
+  } else if (use_tc(M, d, I, tile_T) && use_layer(M, d, I, tile_T, *dev)) {
+    e = launch_tc_layer(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out,
+                        layer_workspace(workspace, L), *dev, s);
   } else if (use_tc(M, d, I, tile_T)) {
     const TcWorkspace tw = tc_workspace(workspace, L);
     e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, out, residual, tw,

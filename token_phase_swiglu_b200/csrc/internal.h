@@ -21,18 +21,22 @@ cudaError_t current_device_info(const DeviceInfo** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 // The first 256 bytes are control words: the device status word at 0, and
-// the fused kernel's counters: out shares set at 64, finished CTAs at 128,
-// arrival tickets at 192.  They must read zero when a call starts and every
+// the single-launch kernels' counters: set-up shares done at 64, finished
+// CTAs at 128, arrival tickets at 192, and for the tensor-core layer kernel
+// gate-up tiles finished at 224 and operand shares written at 240.  They must read zero when a call starts and every
 // call (a timed-out one too) leaves them at zero, so one workspace serves
 // calls of any M, d and I that fit in it.
 struct WorkspaceLayout {
   size_t status = 0;     // uint32 device status word
-  size_t inited = 64;    // uint32 out shares set (fused kernel)
-  size_t done = 128;     // uint32 finished-CTA counter (fused kernel)
-  size_t ticket = 192;   // uint32 CTA arrival tickets (fused kernel)
+  size_t inited = 64;    // uint32 out shares set (fused kernels)
+  size_t done = 128;     // uint32 finished-CTA counter (fused kernels)
+  size_t ticket = 192;   // uint32 CTA arrival tickets (fused kernels)
+  size_t gu_done = 224;  // uint32 gate-up tiles finished (tensor-core layer kernel)
+  size_t hl_done = 240;  // uint32 operand shares written (tensor-core layer kernel)
   size_t zero_end = 256;
   size_t a = 0;          // bf16 [M x I] intermediate
   size_t b_hl = 0, rinv = 0, partials = 0, counters = 0;  // tensor-core path
+  size_t a_ready = 0;    // tensor-core layer kernel: per gate-up tile flags
   size_t ncounters = 0;
   size_t total = 0;
 };
@@ -96,6 +100,29 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
                              const void* P, int T, int64_t d, int64_t I, void* a,
                              float* out_init, const void* residual, const TcWorkspace& ws,
                              const DeviceInfo& dev, cudaStream_t stream);
+// One-launch tensor-core layer (csrc/layer.cu) for 1 <= M <= 64 token rows:
+// the whole block in one persistent kernel (gate-up stream-K range, then the
+// down stream-K range, per CTA).
+struct LayerWorkspace {
+  void* b_hl;          // bf16 [2 Mt x d] hi/lo operand of x*gamma
+  void* a;             // bf16 [M x I] intermediate
+  float* rinv;         // [M] 1/RMS
+  float* partials;     // stream-K partial accumulators
+  uint32_t* counters;  // per gate-up tile arrival counters
+  int ncounters;
+  uint32_t* a_ready;   // per gate-up tile: its k-block of a is written
+  uint32_t *ticket, *inited, *done, *gu_done, *hl_done, *status;  // control words
+};
+struct LayerSizes {
+  size_t b_hl = 0, rinv = 0, partials = 0, counters = 0, a_ready = 0;
+};
+LayerSizes layer_sizes(int64_t M, int64_t d, int64_t I, int sm_count);
+bool layer_supported(int64_t M, int64_t d, int64_t I, int T, const DeviceInfo& dev);
+cudaError_t launch_tc_layer(const void* x, int64_t M, const void* gamma, float eps,
+                            const void* P, int T, const void* W_down, int64_t d, int64_t I,
+                            const void* residual, float* out, const LayerWorkspace& ws,
+                            const DeviceInfo& dev, cudaStream_t stream);
+
 // out = residual or zero (for a down GEMM with no gate-up prologue before it).
 cudaError_t launch_out_init(float* out, const void* residual, int64_t M, int64_t d,
                             const DeviceInfo& dev, cudaStream_t stream);

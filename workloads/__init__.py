@@ -50,14 +50,18 @@ class Workload:
 
 
 # The five workload families (token count M, hidden d, intermediate I).
+# `layers` independent layers (own weights each) run back to back in one
+# step, as a model's layers do: the Phi-3-mini model's 32, and a slice of 4
+# (8B) or 2 (70B) layers of the others, so that every workload measures
+# layers that follow each other on the GPU rather than one layer per launch.
 WORKLOADS = {
     "tiny": Workload("tiny", 4, 256, 688, 0.02),
     "phi3_decode": Workload("phi3_decode", 1, 3072, 8192, 0.02, layers=32),
-    "llama8b_decode_m1": Workload("llama8b_decode_m1", 1, 4096, 14336, 0.02),
-    "llama8b_decode_m8": Workload("llama8b_decode_m8", 8, 4096, 14336, 0.02),
-    "llama8b_decode_m32": Workload("llama8b_decode_m32", 32, 4096, 14336, 0.02),
-    "llama70b_verify": Workload("llama70b_verify", 128, 8192, 28672, 0.01),
-    "llama8b_prefill": Workload("llama8b_prefill", 2048, 4096, 14336, 0.02),
+    "llama8b_decode_m1": Workload("llama8b_decode_m1", 1, 4096, 14336, 0.02, layers=4),
+    "llama8b_decode_m8": Workload("llama8b_decode_m8", 8, 4096, 14336, 0.02, layers=4),
+    "llama8b_decode_m32": Workload("llama8b_decode_m32", 32, 4096, 14336, 0.02, layers=4),
+    "llama70b_verify": Workload("llama70b_verify", 128, 8192, 28672, 0.01, layers=2),
+    "llama8b_prefill": Workload("llama8b_prefill", 2048, 4096, 14336, 0.02, layers=2),
 }
 
 
