@@ -130,17 +130,27 @@ def gated_mlp(h, W_gate, W_up, W_down, intermediate=None) -> np.ndarray:
 
 
 def fused_mlp(x, gamma, eps, W_gate, W_up, W_down, residual=None,
-              intermediate=None) -> np.ndarray:
+              intermediate=None, output=None) -> np.ndarray:
     """The whole MLP block: RMSNorm -> Eq(1) -> optional residual add.
 
     [FastTPS] MLP execution flow: RMSNorm -> gate-up -> siLu_Mul -> down
     projection.  ``residual`` (same shape as the output) is added after the
     down projection when given.
+
+    ``output='bf16'`` returns the block's result rounded once to bf16 (round
+    to nearest, ties to even) after the residual add: the output that the
+    next layer reads as its input when layers are chained in bf16 (the bf16
+    simulation of [FastTPS] section 六 keeps tensors between operators in
+    bf16).  The default returns the binary64 result.
     """
     h = rmsnorm(x, gamma, eps)
     O = gated_mlp(h, W_gate, W_up, W_down, intermediate=intermediate)
     if residual is not None:
         O = O + np.asarray(residual, dtype=np.float64)
+    if output == "bf16":
+        O = round_to_bf16(O)
+    elif output is not None:
+        raise ValueError(f"unknown output precision {output!r}")
     return O
 
 
@@ -192,19 +202,19 @@ def unpack_gate_up(P, I: int, T: int):
 
 
 def fused_mlp_packed(x, gamma, eps, P, T, W_down, residual=None,
-                     intermediate=None) -> np.ndarray:
+                     intermediate=None, output=None) -> np.ndarray:
     """The MLP block with gate/up weights read from the packed matrix P."""
     I = np.asarray(P).shape[0] // 2
     Wg, Wu = unpack_gate_up(P, I, T)
     return fused_mlp(x, gamma, eps, Wg, Wu, W_down, residual=residual,
-                     intermediate=intermediate)
+                     intermediate=intermediate, output=output)
 
 
 def fused_mlp_bf16(x_bits, gamma_bits, eps, Wg_bits, Wu_bits, Wd_bits,
-                   residual_bits=None, intermediate=None) -> np.ndarray:
+                   residual_bits=None, intermediate=None, output=None) -> np.ndarray:
     """``fused_mlp`` fed bf16 bit patterns (the same bytes the GPU reads),
     each decoded exactly to binary64 first."""
     res = None if residual_bits is None else decode_bf16(residual_bits)
     return fused_mlp(decode_bf16(x_bits), decode_bf16(gamma_bits), float(eps),
                      decode_bf16(Wg_bits), decode_bf16(Wu_bits), decode_bf16(Wd_bits),
-                     residual=res, intermediate=intermediate)
+                     residual=res, intermediate=intermediate, output=output)

@@ -390,10 +390,12 @@ def test_bounded_wait_timeout_reports_and_recovers(fm):
     word, lets its in-flight copies land and returns; the context stays usable
     and the next call, with injection off, is correct."""
     dev = torch.device("cuda:0")
-    for M in (2, 7):   # the fused kernel, and the tensor-core path
-        p = wl.make_problem(M, 1024, 2048, seed=12)
+    # the CUDA-core fused kernel, the three tensor-core launches, and the
+    # one-launch tensor-core layer (4 rows of a layer above 200 MB)
+    for M, d, I in ((2, 1024, 2048), (7, 1024, 2048), (4, 4096, 8192)):
+        p = wl.make_problem(M, d, I, seed=12)
         g = {k: v.to(dev) for k, v in p.items()}
-        d, I, T = 1024, 2048, 16
+        T = 16
         packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
         fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
         ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)

@@ -327,12 +327,43 @@ def pin_bf16_entry_decodes(o):
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
 
 
+def pin_bf16_output(o):
+    """The bf16 output of the chained block: the binary64 result, residual
+    included, rounded once.  Checked against torch's own binary64 -> bf16
+    conversion of the block's binary64 output (an independent rounding), its
+    half-step error bound, exact bf16 values, and the zero-weight case where
+    the output is the (bf16) residual itself."""
+    rng = np.random.default_rng(11)
+    M, d, I = 3, 64, 48
+    x = _bf16_values(rng, (M, d))
+    gamma = _bf16_values(rng, (d,), 0.1, 1.0)
+    Wg, Wu = _bf16_values(rng, (I, d), 0.2), _bf16_values(rng, (I, d), 0.2)
+    Wd = _bf16_values(rng, (d, I), 0.2)
+    res = _bf16_values(rng, (M, d))
+    for r in (None, res):
+        exact = o.fused_mlp(x, gamma, 1e-5, Wg, Wu, Wd, residual=r)
+        got = o.fused_mlp(x, gamma, 1e-5, Wg, Wu, Wd, residual=r, output="bf16")
+        ref = torch.from_numpy(exact).to(torch.bfloat16).to(torch.float64).numpy()
+        assert np.array_equal(got, ref)
+        # a bf16 value v in [2^(e-1), 2^e) has step 2^(e-8): within half a step
+        step = np.ldexp(1.0, np.frexp(exact)[1] - 8)
+        assert np.all(np.abs(got - exact) <= step / 2)
+        assert np.array_equal(o.round_to_bf16(got), got)
+    # the rounding happens after the residual add, not before it
+    before = o.round_to_bf16(o.fused_mlp(x, gamma, 1e-5, Wg, Wu, Wd)) + res
+    assert not np.array_equal(o.fused_mlp(x, gamma, 1e-5, Wg, Wu, Wd, residual=res,
+                                          output="bf16"), before)
+    # zero gate weights: SiLU(0) = 0, so the output is the residual exactly
+    zero = o.fused_mlp(x, gamma, 1e-5, 0 * Wg, Wu, Wd, residual=res, output="bf16")
+    assert np.array_equal(zero, res)
+
+
 PINS = [pin_decode_bf16_exhaustive, pin_round_to_bf16, pin_rms_inv_vs_norm,
         pin_rmsnorm_scale_invariance, pin_silu, pin_closed_form_d1_I1, pin_zero_invariants,
         pin_bruteforce_tiny, pin_saturated_gate_is_bilinear, pin_swiglu_intermediate,
         pin_intermediate_rounding,
         pin_interleave_golden, pin_interleave_is_permutation, pin_packed_forward_equals_plain,
-        pin_bf16_entry_decodes]
+        pin_bf16_entry_decodes, pin_bf16_output]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -411,6 +442,15 @@ def _mut_round_truncate(v):
     return np.ldexp(np.trunc(np.ldexp(m, 8)), e - 8)
 
 
+def _mut_fused_round_before_residual(x, gamma, eps, W_gate, W_up, W_down, residual=None,
+                                     intermediate=None, output=None):
+    O = ofm._orig_fused_mlp(x, gamma, eps, W_gate, W_up, W_down, intermediate=intermediate,
+                            output=output)
+    if residual is not None:
+        O = O + np.asarray(residual, dtype=np.float64)
+    return O
+
+
 MUTANTS = {
     "silu_sign": ("silu", _mut_silu_sign),
     "silu_is_sigmoid": ("silu", _mut_silu_sigmoid),
@@ -423,6 +463,7 @@ MUTANTS = {
     "gate_up_swapped_in_tile": ("interleaved_rows", _mut_interleave_swapped),
     "no_interleave": ("interleaved_rows", _mut_interleave_plain_concat),
     "bf16_truncates": ("round_to_bf16", _mut_round_truncate),
+    "output_rounded_before_residual": ("fused_mlp", _mut_fused_round_before_residual),
 }
 
 
@@ -431,6 +472,7 @@ def test_oracle_mutants_are_caught(name, monkeypatch):
     attr, fn = MUTANTS[name]
     monkeypatch.setattr(ofm, "_orig_gated_mlp", ofm.gated_mlp, raising=False)
     monkeypatch.setattr(ofm, "_orig_interleaved_rows", ofm.interleaved_rows, raising=False)
+    monkeypatch.setattr(ofm, "_orig_fused_mlp", ofm.fused_mlp, raising=False)
     monkeypatch.setattr(ofm, attr, fn)
     caught = []
     for pin in PINS:

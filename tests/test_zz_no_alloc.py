@@ -119,10 +119,11 @@ def test_noalloc_matches_oracle_and_workspace_entry_point(cuda_device, M, d, I, 
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("M,d,I", [(2, 1024, 2048), (7, 1024, 2048)])
+@pytest.mark.parametrize("M,d,I", [(2, 1024, 2048), (7, 1024, 2048), (4, 4096, 8192)])
 def test_noalloc_recovers_after_a_timed_out_call(cuda_device, M, d, I):
-    """A call whose bounded waits expire (the fused kernel at M=2, the
-    tensor-core path at M=7) leaves the scratch buffer's control words
+    """A call whose bounded waits expire (the fused CUDA-core kernel at M=2,
+    the three tensor-core launches at M=7, the one-launch tensor-core layer
+    at M=4 on a 201 MB layer) leaves the scratch buffer's control words
     dirty; the next call clears them before its kernels run and is correct."""
     import token_phase_swiglu_b200 as fm
     dev = cuda_device
