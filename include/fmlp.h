@@ -78,10 +78,11 @@ FMLP_API fmlp_status fmlp_pack(const void* W_gate, const void* W_up, int64_t d, 
                       int tile_T, void* packed, void* stream);
 
 /*
- * fmlp_workspace_bytes -- bytes of device workspace fmlp_forward needs for
- * (M, d, I).  The workspace holds a device status word, the fused decode
- * kernel's two completion counters, the bf16 intermediate a [M x I], and
- * the tensor-core path's operand copy and stream-K partials.  A workspace
+ * fmlp_workspace_bytes -- bytes of device workspace fmlp_forward (and
+ * fmlp_forward_bf16) needs for (M, d, I).  The workspace holds a device
+ * status word, the single-launch kernels' counters, the bf16 intermediate
+ * a [M x I], the tensor-core paths' operand copy, stream-K partials and tile
+ * flags, and an f32 [M x d] sum for a bf16 output.  A workspace
  * must be zero-filled before its first use; after that, every call (a
  * timed-out one too) leaves it ready for the next call of any sizes whose
  * fmlp_workspace_bytes it does not exceed.  Returns 0 for invalid sizes.
@@ -137,6 +138,32 @@ FMLP_API fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, f
                          const void* packed_Wgu, int tile_T, const void* W_down,
                          int64_t d, int64_t I, const void* residual, float* out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fmlp_forward_bf16 -- the MLP block with a bf16 output, for chaining layers:
+ *     out = bf16_RN( a W_down^T + residual )
+ * rounded once, after the residual add (round to nearest even), so that the
+ * result can be fed to the next layer as its x.  FastTPS section 三, Eq(1)
+ * and the MLP execution flow as in fmlp_forward; section 六 (bf16 simulation:
+ * the tensors passed between operators are bf16).
+ *
+ * Arguments as in fmlp_forward, except
+ *   out : bf16 [M x d].  It may be the same buffer as x or as residual (an
+ *         in-place update of the residual stream): it is written only after
+ *         every read of them.  It must not overlap the workspace or a weight.
+ * The f32 sum is kept in the workspace (fmlp_workspace_bytes covers it).
+ * Precision: as fmlp_forward up to the f32 sum, then one rounding to bf16;
+ * against the binary64 block the output differs by that rounding (at most
+ * half a bf16 step per element) on top of fmlp_forward's error.
+ *
+ * Kernels: the single-launch paths of fmlp_forward round the sum in their
+ * last thread block to finish (still one launch); the multi-launch paths add
+ * one small rounding launch.
+ */
+FMLP_API fmlp_status fmlp_forward_bf16(const void* x, int64_t M, const void* gamma, float eps,
+                                       const void* packed_Wgu, int tile_T, const void* W_down,
+                                       int64_t d, int64_t I, const void* residual, void* out,
+                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * fmlp_gate_up_swiglu -- steps a1-a4 alone: writes the bf16 intermediate
@@ -196,8 +223,8 @@ FMLP_API fmlp_status fmlp_device_status(void* workspace, void* stream);
  * before anything is enqueued.  Of the benchmarked shapes, the tiny layer
  * (M=4, d=256, I=688), the Phi-3-mini decode layer (M=1, d=3072, I=8192)
  * and the Llama-3.1-8B decode layer at M=1 and M=8 (d=4096, I=14336) fit;
- * the 8B layer at M=32 (11.4 MiB), the 70B verify layer (M=128, 51 MiB)
- * and the 8B prefill chunk (M=2048, 128 MiB) do not.  Each call first clears the buffer's control
+ * the 8B layer at M=32 (11.9 MiB), the 70B verify layer (M=128, 55 MiB)
+ * and the 8B prefill chunk (M=2048, 160 MiB) do not.  Each call first clears the buffer's control
  * words on `stream`, then runs the fmlp_forward kernels on it.  Every call in
  * the process shares the one buffer: calls that may overlap on the GPU (two
  * streams, or two threads) race and must not be issued.  A device-side

@@ -636,3 +636,118 @@ def test_tensor_core_layer_back_to_back_layers(fm):
     refs = {False: oracle_out(p), True: oracle_out(p, residual=True)}
     for i, out in enumerate(outs):
         assert_parity(out.cpu().double().numpy(), refs[bool(i % 3)])
+
+
+# ----------------------------------------------------------------------------
+# bf16 output for chained layers: out = bf16(a W_down^T + residual)
+# ----------------------------------------------------------------------------
+# Bar for this mode (the stated 2e-3 cannot hold once the output itself is
+# rounded): rounding a and the output to bf16 costs 1.7e-3..2.4e-3 normwise
+# against the binary64 block on these workloads (an f32 restatement of the
+# arithmetic, seed 0), so normwise <= 3e-3 and, unchanged, per-element <=
+# 1e-2 max|O_ref|.  Tight: against the oracle with a and the output rounded
+# to bf16, every element within one bf16 step (plus a small absolute term for
+# elements that cancel to near zero) and almost all equal.
+TOL_NORM_BF16OUT = 3e-3
+
+
+def run_forward_bf16(fm, p, T=16, residual=False, alias=None):
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in p.items()}
+    M, d = g["x"].shape
+    I = g["W_gate"].shape[0]
+    packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+    fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    out = {"x": g["x"], "residual": g.get("residual")}.get(alias) if alias else None
+    if out is None:
+        out = torch.full((M, d), float("nan"), dtype=torch.bfloat16, device=dev)
+    launches = fm.fmlp_kernel_launch_count()
+    fm.fmlp_forward_bf16(g["x"], g["gamma"], EPS, packed, T, g["W_down"], out, ws,
+                         residual=g["residual"] if residual else None)
+    launches = fm.fmlp_kernel_launch_count() - launches
+    torch.cuda.synchronize()
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+    return bits(out), launches
+
+
+def assert_parity_bf16out(got_bits, p, residual):
+    got = oracle.decode_bf16(got_bits)
+    ref = oracle_out(p, residual=residual)
+    norm, elem = errors(got, ref)
+    assert norm <= TOL_NORM_BF16OUT, f"normwise {norm:.3e}"
+    assert elem <= TOL_ELEM, f"per-element {elem:.3e}"
+    b = {k: bits(v) for k, v in p.items()}
+    tight = oracle.fused_mlp_bf16(b["x"], b["gamma"], EPS, b["W_gate"], b["W_up"], b["W_down"],
+                                  residual_bits=b["residual"] if residual else None,
+                                  intermediate="bf16", output="bf16")
+    # one bf16 step of the element, plus an absolute 5e-4 max|out| for
+    # elements that cancel to near zero: the sum's error scales with its
+    # terms, not with the small result.  Measured before rounding, the
+    # CUDA-core paths' f32 sums stay within 2e-6 max|out| of this oracle, the
+    # tensor-core paths' within 1.6e-4 at K = 4096 (their accumulation rounds
+    # more coarsely than a sequential f32 sum, so more elements of a flip).
+    step = np.ldexp(1.0, np.frexp(tight)[1] - 8)
+    off = np.abs(got - tight)
+    allowed = step * 1.0001 + 5e-4 * np.max(np.abs(tight))
+    assert np.all(off <= allowed), f"max {np.max(off / allowed):.2f} of the allowance"
+    # measured: 96.4% equal on the tensor-core path at K = 4096
+    assert (off == 0).mean() >= 0.90, f"only {(off == 0).mean():.3f} equal"
+    return norm
+
+
+@pytest.mark.parametrize("M,d,I,T,launches", [
+    (1, 3072, 8192, 16, 1),      # CUDA-core fused kernel, last block rounds
+    (3, 1024, 2064, 16, 1),      # CUDA-core fused kernel, 3 rows
+    (8, 4096, 8192, 16, 1),      # one-launch tensor-core layer, last block rounds
+    (24, 512, 1024, 16, 4),      # three tensor-core launches + the rounding launch
+    (9, 256, 688, 8, 3),         # streaming kernels (I % 64 != 0) + the rounding launch
+])
+def test_bf16_output_every_path(fm, M, d, I, T, launches):
+    p = wl.make_problem(M, d, I, sigma=0.02, seed=60 + M, residual=True)
+    for residual in (False, True):
+        got, n = run_forward_bf16(fm, p, T=T, residual=residual)
+        assert n == launches
+        assert_parity_bf16out(got, p, residual)
+
+
+@pytest.mark.parametrize("alias", ["x", "residual"])
+@pytest.mark.parametrize("M,d,I", [(1, 3072, 8192), (8, 4096, 8192), (24, 512, 1024)])
+def test_bf16_output_in_place(fm, M, d, I, alias):
+    """out may be x itself or the residual itself (the residual stream updated
+    in place): it is written after every read of them."""
+    p = wl.make_problem(M, d, I, sigma=0.02, seed=70 + M, residual=True)
+    got, _ = run_forward_bf16(fm, p, residual=True, alias=alias)
+    assert_parity_bf16out(got, p, True)
+
+
+def test_bf16_output_chained_layers(fm):
+    """Three layers chained through the bf16 output, each fed the previous
+    layer's output as x and as residual (pre-norm residual stream): every
+    layer matches the oracle fed the same bf16 bytes."""
+    dev = torch.device("cuda:0")
+    M, d, I, T = 8, 4096, 8192, 16
+    x = wl.make_activations(M, d, seed=80)["x"].to(dev)
+    ws = torch.zeros(fm.fmlp_workspace_bytes(M, d, I), dtype=torch.uint8, device=dev)
+    for layer in range(3):
+        w = wl.make_weights(d, I, 0.02, seed=81 + layer)
+        gamma = wl.normal_bf16(81 + layer, wl.TID_GAMMA, (d,), mean=1.0, std=0.1)
+        g = {k: v.to(dev) for k, v in w.items()}
+        packed = torch.empty(2 * I, d, dtype=torch.bfloat16, device=dev)
+        fm.fmlp_pack(g["W_gate"], g["W_up"], T, packed)
+        x_in = x.clone()
+        fm.fmlp_forward_bf16(x, gamma.to(dev), EPS, packed, T, g["W_down"], x, ws, residual=x)
+        torch.cuda.synchronize()
+        p = {"x": x_in.cpu(), "gamma": gamma, "residual": x_in.cpu(), **w}
+        assert_parity_bf16out(bits(x), p, True)
+    assert fm.fmlp_device_status(ws) == fm.FMLP_OK
+
+
+@pytest.mark.parametrize("name", ["phi3_decode", "llama8b_decode_m1", "llama8b_decode_m8",
+                                  "llama8b_decode_m32"])
+def test_bf16_output_full_size(fm, name):
+    w = wl.WORKLOADS[name]
+    p = wl.make_problem(w.M, w.d, w.I, sigma=w.sigma, seed=3, residual=True)
+    got, _ = run_forward_bf16(fm, p, residual=True)
+    norm = assert_parity_bf16out(got, p, True)
+    print(f"{name} bf16 output: normwise {norm:.3e}")

@@ -20,7 +20,7 @@ __all__ = [
     "FMLP_ERR_TIMEOUT", "LIB_PATH", "lib", "fmlp_pack", "fmlp_workspace_bytes", "fmlp_forward",
     "fmlp_gate_up_swiglu", "fmlp_down_proj", "fmlp_device_status", "fmlp_status_string",
     "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "fmlp_set_wait_timeout_ns", "fmlp_set_fault_injection",
-    "fmlp_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "fmlp_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "fmlp_forward_bf16",
 ]
 
 FMLP_OK, FMLP_ERR_INVALID_ARG, FMLP_ERR_UNSUPPORTED, FMLP_ERR_CUDA, FMLP_ERR_TIMEOUT = range(5)
@@ -43,6 +43,7 @@ _SIGNATURES = {
     "fmlp_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
     "fmlp_set_fault_injection": (None, [_int]),
     "fmlp_forward_noalloc": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp]),
+    "fmlp_forward_bf16": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -213,6 +214,23 @@ def fmlp_forward(x, gamma, eps: float, packed, tile_T: int, W_down, out, workspa
                                    _ptr(W_down), d, I, _ptr(residual), _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)),
                   "fmlp_forward")
+
+
+def fmlp_forward_bf16(x, gamma, eps: float, packed, tile_T: int, W_down, out, workspace,
+                      residual=None, stream=None) -> None:
+    """out [M x d] (bf16) <- bf16(RMSNorm + gated MLP of x + residual): the output
+    chained layers feed to each other.  out may be x or residual itself."""
+    M, d, I = _check_forward_args(x, gamma, packed, W_down, out, residual)
+    _check(out, "out", torch.bfloat16, (M, d))
+    _check_workspace(workspace, fmlp_workspace_bytes(M, d, I))
+    _on_device(x=x, gamma=gamma, packed=packed, W_down=W_down, residual=residual, out=out,
+               workspace=workspace)
+    _check_status(lib.fmlp_forward_bf16(_ptr(x), M, _ptr(gamma), eps, _ptr(packed), tile_T,
+                                        _ptr(W_down), d, I, _ptr(residual), _ptr(out),
+                                        _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)),
+                  "fmlp_forward_bf16")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20   # FMLP_NOALLOC_SCRATCH_BYTES in include/fmlp.h

@@ -167,6 +167,9 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I) {
     L.a_ready = off;
     off += align256(zl.a_ready);
   }
+  // the f32 sum of a call with a bf16 output (fmlp_forward_bf16)
+  L.out_acc = off;
+  off += align256((size_t)M * (size_t)d * 4);
   L.total = off;
   return L;
 }
@@ -281,14 +284,17 @@ fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down, int64_t
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
 }
 
-fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
-                         const void* packed_Wgu, int tile_T, const void* W_down, int64_t d,
-                         int64_t I, const void* residual, float* out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+// The MLP block into out (f32), or, with out_bf16 set, into the workspace's
+// f32 sum and then rounded to out_bf16.
+static fmlp_status forward_impl(const void* x, int64_t M, const void* gamma, float eps,
+                                const void* packed_Wgu, int tile_T, const void* W_down,
+                                int64_t d, int64_t I, const void* residual, float* out,
+                                void* out_bf16, void* workspace, size_t workspace_bytes,
+                                void* stream) {
   fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
   if (st != FMLP_OK) return st;
   if (!gamma || !packed_Wgu || !W_down) return FMLP_ERR_INVALID_ARG;
-  if (M > 0 && (!x || !out)) return FMLP_ERR_INVALID_ARG;
+  if (M > 0 && (!x || (!out && !out_bf16))) return FMLP_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed_Wgu) || !aligned16(W_down) ||
       !aligned16(out) || !aligned16(residual))
     return FMLP_ERR_INVALID_ARG;
@@ -301,16 +307,20 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
   void* a = (char*)workspace + L.a;
   uint32_t* status = status_word(workspace);
   cudaStream_t s = (cudaStream_t)stream;
+  if (out_bf16) out = (float*)((char*)workspace + L.out_acc);
   cudaError_t e;
+  bool rounded = false;  // the kernel rounded out to out_bf16 itself
   if (!use_tc(M, d, I, tile_T) && fused_decode_supported(M, d, I, *dev)) {
     uint32_t* ticket = (uint32_t*)((char*)workspace + L.ticket);
     uint32_t* inited = (uint32_t*)((char*)workspace + L.inited);
     uint32_t* done = (uint32_t*)((char*)workspace + L.done);
     e = launch_fused_decode(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out,
-                            ticket, inited, done, status, *dev, s);
+                            out_bf16, ticket, inited, done, status, *dev, s);
+    rounded = true;
   } else if (use_tc(M, d, I, tile_T) && use_layer(M, d, I, tile_T, *dev)) {
     e = launch_tc_layer(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out,
-                        layer_workspace(workspace, L), *dev, s);
+                        out_bf16, layer_workspace(workspace, L), *dev, s);
+    rounded = true;
   } else if (use_tc(M, d, I, tile_T)) {
     const TcWorkspace tw = tc_workspace(workspace, L);
     e = launch_tc_gateup(x, M, gamma, eps, packed_Wgu, tile_T, d, I, a, out, residual, tw,
@@ -321,7 +331,33 @@ fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
     if (e == cudaSuccess)
       e = launch_down_stream(a, M, W_down, d, I, residual, out, status, *dev, s);
   }
+  if (e == cudaSuccess && out_bf16 && !rounded) e = launch_out_bf16(out, out_bf16, M, d, *dev, s);
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
+fmlp_status fmlp_forward(const void* x, int64_t M, const void* gamma, float eps,
+                         const void* packed_Wgu, int tile_T, const void* W_down, int64_t d,
+                         int64_t I, const void* residual, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return forward_impl(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, out,
+                      nullptr, workspace, workspace_bytes, stream);
+}
+
+fmlp_status fmlp_forward_bf16(const void* x, int64_t M, const void* gamma, float eps,
+                              const void* packed_Wgu, int tile_T, const void* W_down, int64_t d,
+                              int64_t I, const void* residual, void* out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (M > 0 && !out) return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(out)) return FMLP_ERR_INVALID_ARG;
+  // out may be x or the residual itself (it is written after every read of
+  // them), but must not overlap the workspace
+  if (M > 0) {
+    const uintptr_t o0 = (uintptr_t)out, o1 = o0 + (uintptr_t)(M * d * 2);
+    const uintptr_t w0 = (uintptr_t)workspace, w1 = w0 + workspace_bytes;
+    if (workspace && o0 < w1 && w0 < o1) return FMLP_ERR_INVALID_ARG;
+  }
+  return forward_impl(x, M, gamma, eps, packed_Wgu, tile_T, W_down, d, I, residual, nullptr,
+                      out, workspace, workspace_bytes, stream);
 }
 
 fmlp_status fmlp_device_status(void* workspace, void* stream) {

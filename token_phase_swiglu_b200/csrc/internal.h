@@ -37,6 +37,7 @@ struct WorkspaceLayout {
   size_t a = 0;          // bf16 [M x I] intermediate
   size_t b_hl = 0, rinv = 0, partials = 0, counters = 0;  // tensor-core path
   size_t a_ready = 0;    // tensor-core layer kernel: per gate-up tile flags
+  size_t out_acc = 0;    // f32 [M x d] sum of a call with a bf16 output
   size_t ncounters = 0;
   size_t total = 0;
 };
@@ -73,11 +74,12 @@ cudaError_t launch_gateup_stream(const void* x, int64_t M, const void* gamma, fl
 // workspace's counters of arrivals, of out shares set and of CTAs finished,
 // zero on entry and on exit.
 bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& dev);
+// out_bf16 (or null): the last CTA to finish rounds out to it.
 cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                                const void* residual, float* out, uint32_t* ticket,
-                                uint32_t* inited, uint32_t* done, uint32_t* status,
-                                const DeviceInfo& dev, cudaStream_t stream);
+                                const void* residual, float* out, void* out_bf16,
+                                uint32_t* ticket, uint32_t* inited, uint32_t* done,
+                                uint32_t* status, const DeviceInfo& dev, cudaStream_t stream);
 
 // Tensor-core path (tcgen05, csrc/tc.cu) for M above the decode range.
 constexpr int kTcMaxCtas = 160;  // workspace sizing bound on the grid (>= SMs of a B200)
@@ -120,7 +122,11 @@ LayerSizes layer_sizes(int64_t M, int64_t d, int64_t I, int sm_count);
 bool layer_supported(int64_t M, int64_t d, int64_t I, int T, const DeviceInfo& dev);
 cudaError_t launch_tc_layer(const void* x, int64_t M, const void* gamma, float eps,
                             const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                            const void* residual, float* out, const LayerWorkspace& ws,
+                            const void* residual, float* out, void* out_bf16,
+                            const LayerWorkspace& ws, const DeviceInfo& dev,
+                            cudaStream_t stream);
+// dst (bf16 [M x d]) = src (f32) rounded, after the previous kernel on the stream.
+cudaError_t launch_out_bf16(const float* src, void* dst, int64_t M, int64_t d,
                             const DeviceInfo& dev, cudaStream_t stream);
 
 // out = residual or zero (for a down GEMM with no gate-up prologue before it).

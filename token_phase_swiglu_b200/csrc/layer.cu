@@ -83,7 +83,8 @@ struct LayerParams {
   const __nv_bfloat16* residual;
   __nv_bfloat16* b_hl; // [2 Mt x d]: rows [0, Mt) hi(x*gamma), [Mt, 2 Mt) lo
   __nv_bfloat16* a;    // [M x I] intermediate
-  float* out;          // [M x d]
+  float* out;          // [M x d] f32 sum (set to the residual or zero, then added into)
+  __nv_bfloat16* out_bf16;  // [M x d] or null: out rounded to bf16 by the last CTA to finish
   float* rinv;         // [M]
   float* partials;     // [ctas][2][2 Mt][128]
   uint32_t* counters;  // gate-up tile arrivals [tiles_g]
@@ -126,6 +127,7 @@ struct LayerShared {
   int kb_issued;       // stages whose activations the loader issued
   uint32_t ticket;
   int ready;           // epilogue: set-up shares seen (1) or gave up (-1)
+  int last_cta;        // this CTA was the last to finish
   float rinv_s[kLayerMaxMt];
 };
 
@@ -688,6 +690,9 @@ __global__ void __launch_bounds__(kLayerThreads, 1) tc_layer(const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.acc_empty[buf]);
     }
+    // with a bf16 output the last CTA to finish reads the sum: this thread's
+    // adds into it are visible before its CTA counts itself finished
+    if (p.out_bf16) __threadfence();
   } else {
     // ---------------- activation loader (warp 6) ----------------
     if (lane == 0) {
@@ -752,17 +757,31 @@ __global__ void __launch_bounds__(kLayerThreads, 1) tc_layer(const __grid_consta
         mbar_wait_bounded(&sh.full[k % p.stages], (uint32_t)((k / p.stages) & 1),
                           kLayerDrainNs, nullptr);
     }
+    // this CTA's adds into out are visible before it counts itself finished
+    if (p.out_bf16) __threadfence();
     // Every CTA took its ticket, wrote its shares and finished its waits on
     // the counters: the last one here leaves them at zero for the next call.
-    if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+    const bool last = atomicAdd(p.done, 1u) == gridDim.x - 1;
+    if (last) {
       atomicExch(p.ticket, 0u);
       atomicExch(p.inited, 0u);
       atomicExch(p.gu_done, 0u);
       atomicExch(p.hl_done, 0u);
       atomicExch(p.done, 0u);
     }
+    sh.last_cta = last;
   }
   __syncthreads();
+  if (p.out_bf16 && sh.last_cta) {
+    // the last CTA rounds the finished sum to the bf16 output
+    __threadfence();
+    const int64_t n4 = (int64_t)p.M * p.d / 4;
+    for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(p.out) + i);
+      reinterpret_cast<uint2*>(p.out_bf16)[i] =
+          make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);
@@ -861,8 +880,9 @@ LayerSizes layer_sizes(int64_t M, int64_t d, int64_t I, int sm_count) {
 
 cudaError_t launch_tc_layer(const void* x, int64_t M, const void* gamma, float eps,
                             const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                            const void* residual, float* out, const LayerWorkspace& ws,
-                            const DeviceInfo& dev, cudaStream_t stream) {
+                            const void* residual, float* out, void* out_bf16,
+                            const LayerWorkspace& ws, const DeviceInfo& dev,
+                            cudaStream_t stream) {
   LayerPlan pl;
   if (!make_layer_plan(M, dev.max_smem_optin, pl)) return cudaErrorInvalidValue;
   cudaError_t e = allow_layer_smem(dev);
@@ -908,6 +928,7 @@ cudaError_t launch_tc_layer(const void* x, int64_t M, const void* gamma, float e
   p.b_hl = (__nv_bfloat16*)ws.b_hl;
   p.a = (__nv_bfloat16*)ws.a;
   p.out = out;
+  p.out_bf16 = (__nv_bfloat16*)out_bf16;
   p.rinv = ws.rinv;
   p.partials = ws.partials;
   p.counters = ws.counters;

@@ -147,6 +147,7 @@ struct CtaState {
   int abort;
   int issued;     // stages issued by the producer
   int out_ready;  // fused_decode: 0 until every share of out is set, then 1 (-1: gave up)
+  int last;       // fused_decode: this CTA was the last to finish
 };
 
 __device__ __forceinline__ void init_ring(const Ring& r, CtaState& st) {
@@ -661,6 +662,7 @@ struct FusedParams {
   const __nv_bfloat16* gamma;
   const __nv_bfloat16* residual;
   float* out;          // [M x d] f32: set to the residual (or 0), then CTAs add into it
+  __nv_bfloat16* out_bf16;  // [M x d] or null: out rounded to bf16 by the last CTA to finish
   uint32_t* ticket;    // arrival order of the CTAs (zero between calls)
   uint32_t* inited;    // initialising CTAs whose share of out is set (zero between calls)
   uint32_t* done;      // CTAs finished (zero between calls)
@@ -790,6 +792,18 @@ __device__ bool wait_counter(const uint32_t* ctr, uint32_t target, uint64_t limi
   }
 }
 
+// The block's threads round n f32 values (n % 4 == 0, read from L2, where
+// other blocks' adds landed) to bf16, round to nearest even.
+__device__ void out_to_bf16_block(const float* src, __nv_bfloat16* dst, int64_t n) {
+  for (int64_t i = threadIdx.x; i < n / 4; i += blockDim.x) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(src) + i);
+    uint2 w;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w.x) : "f"(v.y), "f"(v.x));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w.y) : "f"(v.w), "f"(v.z));
+    reinterpret_cast<uint2*>(dst)[i] = w;
+  }
+}
+
 // Warp 0, lanes 1-31.  The first n_init CTAs to arrive (an atomic ticket,
 // taken once the previous kernel on the stream is done) set one share each
 // of out (float4 granules) to the residual or zero and count it in inited.
@@ -889,17 +903,32 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode(const __grid_constan
       named_barrier_sync(kBarStage, kConsumers * 32);  // slice of a complete
       consume_down_slice<MT>(cs, p, slice, w, mt);
     }
+    // with a bf16 output the last CTA to finish reads the sum: this thread's
+    // adds into it are visible before its CTA counts itself finished
+    if (p.out_bf16) __threadfence();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     if (st.abort) drain_ring(ring, st.issued);
+    // this CTA's adds into out are visible before it counts itself finished
+    if (p.out_bf16) __threadfence();
     // Every CTA has taken its ticket, finished any share of out it owned and
     // is past its wait on `inited`: the last one to get here leaves the
     // counters at zero for the next call (also after a timeout).
-    if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+    const bool last = atomicAdd(p.done, 1u) == gridDim.x - 1;
+    if (last) {
       atomicExch(p.ticket, 0u);
       atomicExch(p.inited, 0u);
       atomicExch(p.done, 0u);
+    }
+    st.last = last;
+  }
+  if (p.out_bf16) {
+    // the last CTA rounds the finished sum to the bf16 output
+    __syncthreads();
+    if (st.last) {
+      __threadfence();
+      out_to_bf16_block(p.out, p.out_bf16, (int64_t)min(MT, p.M) * p.d);
     }
   }
 }
@@ -1147,9 +1176,9 @@ bool fused_decode_supported(int64_t M, int64_t d, int64_t I, const DeviceInfo& d
 
 cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, float eps,
                                 const void* P, int T, const void* W_down, int64_t d, int64_t I,
-                                const void* residual, float* out, uint32_t* ticket,
-                                uint32_t* inited, uint32_t* done, uint32_t* status,
-                                const DeviceInfo& dev, cudaStream_t stream) {
+                                const void* residual, float* out, void* out_bf16,
+                                uint32_t* ticket, uint32_t* inited, uint32_t* done,
+                                uint32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
   const FusedPlan f = make_fused_plan(M, d, I, dev);
   if (f.mt == 0) return cudaErrorInvalidConfiguration;
   FusedParams p;
@@ -1162,6 +1191,7 @@ cudaError_t launch_fused_decode(const void* x, int64_t M, const void* gamma, flo
   p.gamma = (const __nv_bfloat16*)gamma;
   p.residual = (const __nv_bfloat16*)residual;
   p.out = out;
+  p.out_bf16 = (__nv_bfloat16*)out_bf16;
   p.ticket = ticket;
   p.inited = inited;
   p.done = done;

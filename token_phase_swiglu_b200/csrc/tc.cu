@@ -1004,6 +1004,23 @@ __global__ void __launch_bounds__(256) act_split(const __nv_bfloat16* __restrict
   }
 }
 
+// dst = bf16(src), round to nearest even: the f32 sum of the block rounded to
+// its bf16 output once the down projection has finished adding into it.
+__global__ void __launch_bounds__(256) out_bf16_kernel(const float* __restrict__ src,
+                                                       __nv_bfloat16* __restrict__ dst,
+                                                       int64_t n4) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // the sum is complete once the previous kernel is
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(src)[i];
+    uint2 w;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w.x) : "f"(v.y), "f"(v.x));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w.y) : "f"(v.w), "f"(v.z));
+    reinterpret_cast<uint2*>(dst)[i] = w;
+  }
+}
+
 // out = residual (or zero), before a down GEMM that is not preceded by the
 // gate-up prologue (fmlp_down_proj).
 __global__ void __launch_bounds__(256) out_init(float* __restrict__ out,
@@ -1242,6 +1259,24 @@ cudaError_t launch_tc_gateup(const void* x, int64_t M, const void* gamma, float 
   p.rinv = ws.rinv;
   p.a_out = (__nv_bfloat16*)a;
   return launch_tc(p, pl, dev, stream);
+}
+
+cudaError_t launch_out_bf16(const float* src, void* dst, int64_t M, int64_t d,
+                            const DeviceInfo& dev, cudaStream_t stream) {
+  const int64_t n4 = M * d / 4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256,
+                                                                       4 * dev.sm_count)));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, out_bf16_kernel, src, (__nv_bfloat16*)dst, n4);
+  if (e == cudaSuccess) note_launches(1);
+  return e;
 }
 
 cudaError_t launch_out_init(float* out, const void* residual, int64_t M, int64_t d,
