@@ -72,7 +72,8 @@ def measured_peaks() -> dict:
 # when any of them changes)
 KERNEL_SOURCES = {
     "fused_decode": ["stream.cu", "common.cuh", "internal.h"],
-    "tc_gemm": ["tc.cu", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
+    "tc_gemm": ["tc.cu", "tcgen05.cuh", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
+    "tc_layer": ["layer.cu", "tcgen05.cuh", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
 }
 
 

@@ -192,6 +192,32 @@ FMLP_API fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down
                            size_t workspace_bytes, void* stream);
 
 /*
+ * fmlp_sum_partials -- the reduction of a tensor-parallel MLP block:
+ *     out = sum_r partials[r] (+ residual)
+ * When the intermediate dimension I is split over n ranks (each rank holding
+ * whole interleave tiles of packed_Wgu and the matching columns of W_down),
+ * each rank's fmlp_forward with residual = NULL gives a partial output, and
+ * the block's output is their sum: Eq(1) is linear in the columns of a
+ * (FastTPS section 三), and the tensor-parallel layers of "Together AI 的推测
+ * 解码内核融合优化" (blog.hotdry.top) reduce the partial outputs across GPUs
+ * before the next norm.
+ *
+ *   partials  : host array of n device pointers, each f32 [M x d].  A pointer
+ *               may address another GPU's memory mapped into this one (peer
+ *               access); it is read with plain loads, in rank order, so every
+ *               rank computing the sum gets the same bits.
+ *   n         : 1..16
+ *   residual  : bf16 [M x d] added once, or NULL
+ *   out       : f32 [M x d] (out_bf16 == 0) or bf16 [M x d] (out_bf16 != 0,
+ *               rounded once, to nearest even).  An f32 out may be one of the
+ *               partials itself; otherwise it must not overlap them.
+ * Runs after the previous work on `stream` (which wrote the partials).
+ */
+FMLP_API fmlp_status fmlp_sum_partials(const float* const* partials, int n, int64_t M, int64_t d,
+                                       const void* residual, void* out, int out_bf16,
+                                       void* stream);
+
+/*
  * fmlp_device_status -- synchronise `stream`, read the device status word in
  * `workspace` and reset it to zero.  Returns FMLP_ERR_TIMEOUT if a kernel
  * gave up a bounded wait since the last check, FMLP_OK otherwise (or

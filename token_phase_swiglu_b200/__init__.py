@@ -21,6 +21,7 @@ __all__ = [
     "fmlp_gate_up_swiglu", "fmlp_down_proj", "fmlp_device_status", "fmlp_status_string",
     "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "fmlp_set_wait_timeout_ns", "fmlp_set_fault_injection",
     "fmlp_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "fmlp_forward_bf16",
+    "fmlp_sum_partials",
 ]
 
 FMLP_OK, FMLP_ERR_INVALID_ARG, FMLP_ERR_UNSUPPORTED, FMLP_ERR_CUDA, FMLP_ERR_TIMEOUT = range(5)
@@ -44,6 +45,7 @@ _SIGNATURES = {
     "fmlp_set_fault_injection": (None, [_int]),
     "fmlp_forward_noalloc": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp]),
     "fmlp_forward_bf16": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "fmlp_sum_partials": (_int, [ctypes.POINTER(_vp), _int, _i64, _i64, _vp, _vp, _int, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -231,6 +233,25 @@ def fmlp_forward_bf16(x, gamma, eps: float, packed, tile_T: int, W_down, out, wo
                                         workspace.numel() * workspace.element_size(),
                                         _stream(stream)),
                   "fmlp_forward_bf16")
+
+
+def fmlp_sum_partials(partials, out, residual=None, stream=None) -> None:
+    """out [M x d] <- sum of the f32 partial outputs [M x d] (+ residual), out f32 or
+    bf16: the reduction of a tensor-parallel MLP block (partials may be peer memory)."""
+    if not partials:
+        raise ValueError("at least one partial output is needed")
+    M, d = _dims2(partials[0], "partials[0]")
+    for r, t in enumerate(partials):
+        _check(t, f"partials[{r}]", torch.float32, (M, d))
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"out must be float32 or bfloat16, got {out.dtype}")
+    _check(out, "out", out.dtype, (M, d))
+    _check(residual, "residual", torch.bfloat16, (M, d), optional=True)
+    _on_device(out=out, residual=residual)
+    arr = (_vp * len(partials))(*[t.data_ptr() for t in partials])
+    _check_status(lib.fmlp_sum_partials(arr, len(partials), M, d, _ptr(residual), _ptr(out),
+                                        int(out.dtype == torch.bfloat16), _stream(stream)),
+                  "fmlp_sum_partials")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20   # FMLP_NOALLOC_SCRATCH_BYTES in include/fmlp.h

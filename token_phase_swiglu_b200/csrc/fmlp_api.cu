@@ -360,6 +360,28 @@ fmlp_status fmlp_forward_bf16(const void* x, int64_t M, const void* gamma, float
                       out, workspace, workspace_bytes, stream);
 }
 
+fmlp_status fmlp_sum_partials(const float* const* partials, int n, int64_t M, int64_t d,
+                              const void* residual, void* out, int out_bf16, void* stream) {
+  if (n < 1 || n > kMaxPartials || M < 0 || d <= 0 || d % 8 != 0 || d > kMaxD)
+    return FMLP_ERR_INVALID_ARG;
+  if (M == 0) return FMLP_OK;
+  if (!partials || !out || !aligned16(out) || !aligned16(residual)) return FMLP_ERR_INVALID_ARG;
+  const uintptr_t o0 = (uintptr_t)out, o1 = o0 + (uintptr_t)(M * d * (out_bf16 ? 2 : 4));
+  for (int r = 0; r < n; ++r) {
+    if (!partials[r] || !aligned16(partials[r])) return FMLP_ERR_INVALID_ARG;
+    // out may not overlap a partial, unless it is that partial itself (f32)
+    const uintptr_t p0 = (uintptr_t)partials[r], p1 = p0 + (uintptr_t)(M * d * 4);
+    if (o0 < p1 && p0 < o1 && !(o0 == p0 && !out_bf16)) return FMLP_ERR_INVALID_ARG;
+  }
+  const DeviceInfo* dev = nullptr;
+  fmlp_status st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  cudaError_t e = launch_sum_partials(partials, n, M, d, residual,
+                                      out_bf16 ? nullptr : (float*)out, out_bf16 ? out : nullptr,
+                                      *dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
 fmlp_status fmlp_device_status(void* workspace, void* stream) {
   if (!workspace || !aligned16(workspace)) return FMLP_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;

@@ -129,6 +129,13 @@ cudaError_t launch_tc_layer(const void* x, int64_t M, const void* gamma, float e
 cudaError_t launch_out_bf16(const float* src, void* dst, int64_t M, int64_t d,
                             const DeviceInfo& dev, cudaStream_t stream);
 
+// Sum of n partial outputs (+ residual) into out_f32 and/or out_bf16
+// (csrc/reduce.cu); the partials may be peer pointers.
+constexpr int kMaxPartials = 16;
+cudaError_t launch_sum_partials(const float* const* parts, int n, int64_t M, int64_t d,
+                                const void* residual, float* out_f32, void* out_bf16,
+                                const DeviceInfo& dev, cudaStream_t stream);
+
 // out = residual or zero (for a down GEMM with no gate-up prologue before it).
 cudaError_t launch_out_init(float* out, const void* residual, int64_t M, int64_t d,
                             const DeviceInfo& dev, cudaStream_t stream);
