@@ -22,6 +22,9 @@ llama.cpp PR #29948 paragraph on interleaved gate/up rows):
 
 and the gate/up interleave, a pure permutation of rows at tile granularity.
 
+``quant.py`` restates this build's int8 weight format (the pages name
+quantized weight streaming but give no format) and the block on it.
+
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, exact invariants, brute force on tiny shapes and the page-described
 row order -- never against the CUDA path.  No function here is "parity
@@ -42,4 +45,10 @@ from .fmlp import (  # noqa: F401
     unpack_gate_up,
     fused_mlp_packed,
     fused_mlp_bf16,
+)
+from .quant import (  # noqa: F401
+    GROUP,
+    quantize_rows,
+    dequantize_rows,
+    fused_mlp_q8,
 )
