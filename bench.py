@@ -40,6 +40,8 @@ import workloads as wl  # noqa: E402
 EPS = 1e-5
 TILE_T = 16
 METRIC = "fused-MLP weight-stream GB/s (% B200 HBM peak) and tokens/s per layer at 1 GPU"
+# decode workloads also measured on this library's int8 weights (entries "<name>_q8")
+Q8_WORKLOADS = ["phi3_decode", "llama8b_decode_m1"]
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
@@ -52,6 +54,12 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 def algorithmic_bytes(M: int, d: int, I: int, residual: bool = False) -> int:
     """Bytes the MLP block must move once: weights 6dI, x 2Md, gamma 2d, out 4Md (+ residual 2Md)."""
     return 6 * d * I + 2 * M * d + 2 * d + 4 * M * d + (2 * M * d if residual else 0)
+
+
+def q8_bytes(M: int, d: int, I: int) -> int:
+    """Algorithmic bytes of the block on int8 weights: 3dI int8 weights and one f32
+    scale per 64 of them, x 2Md, gamma 2d, out 4Md."""
+    return 3 * d * I + 3 * d * I // 64 * 4 + 2 * M * d + 2 * d + 4 * M * d
 
 
 def gateup_bytes(M: int, d: int, I: int) -> int:
@@ -316,8 +324,8 @@ class WorkloadRun:
     W_down (+ gamma), the token rows x, one output slice per layer and a
     workspace; step() runs the whole hot path once through the C ABI."""
 
-    def __init__(self, fm, w: wl.Workload, dev, seed0: int, layers: int = 0):
-        self.fm, self.w, self.dev = fm, w, dev
+    def __init__(self, fm, w: wl.Workload, dev, seed0: int, layers: int = 0, quant: bool = False):
+        self.fm, self.w, self.dev, self.quant = fm, w, dev, quant
         self.M, self.d, self.I = w.M, w.d, w.I
         self.L = layers or w.layers
         self.seed0 = seed0
@@ -333,8 +341,18 @@ class WorkloadRun:
             fm.fmlp_pack(wg, wu, TILE_T, packed)
             torch.cuda.synchronize()
             del wg, wu
-            self.layers.append({"packed": packed, "W_down": wts["W_down"].to(dev),
-                                "gamma": gamma, "out": self.outs[l]})
+            layer = {"packed": packed, "W_down": wts["W_down"].to(dev), "gamma": gamma,
+                     "out": self.outs[l]}
+            if quant:   # this library's int8 format of the packed gate/up rows and W_down
+                for k in ("packed", "W_down"):
+                    W = layer.pop(k)
+                    q = torch.empty(W.shape, dtype=torch.int8, device=dev)
+                    sc = torch.empty(W.shape[0], W.shape[1] // fm.Q8_GROUP, dtype=torch.float32,
+                                     device=dev)
+                    fm.fmlp_quantize_q8(W, q, sc)
+                    layer[k + "_q"], layer[k + "_s"] = q, sc
+                torch.cuda.synchronize()
+            self.layers.append(layer)
         self.ws = torch.zeros(fm.fmlp_workspace_bytes(w.M, w.d, w.I), dtype=torch.uint8,
                               device=dev)
         self.stream = torch.cuda.current_stream()
@@ -346,8 +364,12 @@ class WorkloadRun:
         x = self.x if x is None else x
         for li, ly in enumerate(self.layers):
             out = ly["out"] if outs is None else outs[li]
-            fm.fmlp_forward(x, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], out,
-                            self.ws, stream=stream)
+            if self.quant:
+                fm.fmlp_forward_q8(x, ly["gamma"], EPS, ly["packed_q"], ly["packed_s"], TILE_T,
+                                   ly["W_down_q"], ly["W_down_s"], out, self.ws, stream=stream)
+            else:
+                fm.fmlp_forward(x, ly["gamma"], EPS, ly["packed"], TILE_T, ly["W_down"], out,
+                                self.ws, stream=stream)
 
     def capture(self, warmup: int, use_graph: bool = True) -> None:
         """Warm-up from the host (also the library's one-time set-up, before
@@ -531,7 +553,12 @@ def roofline_entry(run: WorkloadRun, ms_step: float, gu_ms, sustained: bool = Fa
     M, d, I, L, w = run.M, run.d, run.I, run.L, run.w
     (peak, peak_src), (tpeak, tpeak_src) = peaks_of(sustained)
     single = run.per_step is not None and run.per_step == L
-    if single:
+    if run.quant:
+        # the int8 path: two launches per layer, both weight streams
+        kname, kms = "q8_gateup + q8_down", ms_step / L
+        timing = "timed region / layers (two launches per layer, back to back in a CUDA graph)"
+        kbytes, kflops = q8_bytes(M, d, I), 6 * M * d * I
+    elif single:
         kname = "fused_decode" if M <= 4 else "tc_layer"
         kms = ms_step / L
         timing = "timed region / launches (the step's only kernel, back to back in a CUDA graph)"
@@ -545,8 +572,9 @@ def roofline_entry(run: WorkloadRun, ms_step: float, gu_ms, sustained: bool = Fa
     else:
         bound, kpeak, src, unit, work = "hbm", peak, peak_src, "GB/s", kbytes
     achieved = work / (kms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
-    traffic = recorded_traffic("fused_decode" if kname == "fused_decode" else
-                               ("tc_layer" if kname == "tc_layer" else "tc_gemm"), w.name)
+    traffic = None if run.quant else recorded_traffic(
+        "fused_decode" if kname == "fused_decode" else
+        ("tc_layer" if kname == "tc_layer" else "tc_gemm"), w.name)
     return {"bound": bound, "kernel": kname, "achieved": round(achieved, 2), "peak": kpeak,
             "peak_source": src, "unit": unit, "frac": round(achieved / kpeak, 4),
             "traffic": traffic, "algorithmic_per_launch": work, "avg_launch_ms": round(kms, 5),
@@ -560,8 +588,14 @@ def oracle_check(run: WorkloadRun, got_outs) -> dict:
     rows = check_rows(w.M)
     b = layer_bits(w, run.seed0, 0)
     import oracle
-    ref = oracle.fused_mlp_bf16(b["x"][rows], b["gamma"], EPS, b["W_gate"], b["W_up"],
-                                b["W_down"])
+    if run.quant:   # the block on the dequantized int8 weights
+        dec = oracle.decode_bf16
+        qs = [oracle.quantize_rows(dec(b[k])) for k in ("W_gate", "W_up", "W_down")]
+        ref = oracle.fused_mlp_q8(dec(b["x"][rows]), dec(b["gamma"]), EPS, *qs[0], *qs[1],
+                                  *qs[2])
+    else:
+        ref = oracle.fused_mlp_bf16(b["x"][rows], b["gamma"], EPS, b["W_gate"], b["W_up"],
+                                    b["W_down"])
     got = got_outs[0].cpu().double().numpy()[rows]
     norm = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
     elem = float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-300))
@@ -570,28 +604,30 @@ def oracle_check(run: WorkloadRun, got_outs) -> dict:
 
 
 def measure_sub_workload(fm, w: wl.Workload, dev, args, barrier, max_over_ranks, rank: int,
-                         world: int) -> dict:
+                         world: int, quant: bool = False) -> dict:
     """One entry of the line's `workloads` object: the workload timed for at
     least --min-seconds of device time, its own clocks, roofline, end-to-end
-    pass and oracle check."""
-    run = WorkloadRun(fm, w, dev, seed0=1000 * rank)
+    pass and oracle check (quant: on this library's int8 weights)."""
+    run = WorkloadRun(fm, w, dev, seed0=1000 * rank, quant=quant)
     run.capture(args.warmup, use_graph=not args.no_graph)
     est = run.step_estimate_ms()
     steps = max(args.steps, int(np.ceil(args.min_seconds * 1e3 / max(est, 1e-3))))
     ms, launches, clocks = run.timed(steps, barrier, max_over_ranks)
     ms_step = ms / steps
     gu_ms = None
-    if not (run.per_step is not None and run.per_step == run.L):
+    if not quant and not (run.per_step is not None and run.per_step == run.L):
         gu_ms = run.isolated_calls(max(3, min(20, steps)), max_over_ranks)["fmlp_gate_up_swiglu_ms"]
     e2e_steps = max(2, min(4000, int(np.ceil(0.5e3 / max(est, 1e-3)))))
     e2e_ms, h2d, d2h = run.e2e(e2e_steps, barrier, max_over_ranks)
-    bytes_step = run.L * algorithmic_bytes(w.M, w.d, w.I)
+    bytes_step = run.L * (q8_bytes(w.M, w.d, w.I) if quant else algorithmic_bytes(w.M, w.d, w.I))
     (peak, _), (tpeak, _) = peaks_of(sustained=True)
     gbs = job_gbs(bytes_step, steps, world, ms)
     tflops = 6 * w.M * w.d * w.I * run.L * steps * world / (ms / 1e3) / 1e12
+    wbytes = run.L * (q8_bytes(w.M, w.d, w.I) - q8_bytes(w.M, w.d, 0) if quant else w.weight_bytes)
     entry = {
         "config": {"M": w.M, "d": w.d, "I": w.I, "layers": run.L, "tile_T": TILE_T,
-                   "weights_per_gpu_GB": round(run.L * w.weight_bytes / 1e9, 3)},
+                   "weights": "int8, one f32 scale per 64 (this library's format)" if quant
+                   else "bf16", "weights_per_gpu_GB": round(wbytes / 1e9, 3)},
         "value": round(gbs, 2), "unit": "GB/s", "hbm_frac": round(gbs / world / peak, 4),
         "tflops": round(tflops, 2), "tensor_frac": round(tflops / world / tpeak, 4),
         "tokens_per_s_per_layer": round(w.M * run.L * steps * world / (ms / 1e3), 1),
@@ -665,10 +701,12 @@ def run_ours(args) -> None:
     # entry each
     subs = {}
     names = [] if args.workloads == "none" else (
-        list(wl.WORKLOADS) if args.workloads == "all" else args.workloads.split(","))
+        list(wl.WORKLOADS) + [n + "_q8" for n in Q8_WORKLOADS] if args.workloads == "all"
+        else args.workloads.split(","))
     for name in names:
-        subs[name] = measure_sub_workload(fm, wl.WORKLOADS[name], dev, args, barrier,
-                                          max_over_ranks, rank, world)
+        quant = name.endswith("_q8")
+        subs[name] = measure_sub_workload(fm, wl.WORKLOADS[name[:-3] if quant else name], dev,
+                                          args, barrier, max_over_ranks, rank, world, quant=quant)
 
     if rank == 0:
         gu_ms, dn_ms = iso["fmlp_gate_up_swiglu_ms"], iso["fmlp_down_proj_ms"]

@@ -192,6 +192,52 @@ FMLP_API fmlp_status fmlp_down_proj(const void* a, int64_t M, const void* W_down
                            size_t workspace_bytes, void* stream);
 
 /*
+ * fmlp_quantize_q8 -- this library's int8 weight format (the pages name
+ * quantized weight streaming over interleaved gate/up rows -- the llama.cpp
+ * PR #29948 paragraph of "CUDAカーネル融合で推論が最大10%高速化",
+ * blog.cecily.jp -- but give no block format).  Each row of W is cut along K
+ * into groups of 64 consecutive elements; group g gets one binary32 scale
+ *     s_g = fl32(max |w| / 127)            (IEEE division, round to nearest)
+ * and each weight the int8
+ *     q = clamp(rint(fl32(w / s_g)), -127, 127)   (rint: halves to even)
+ * (q = 0 in a group of zeros).  The weight stands for q * s_g.  Quantizing
+ * works row by row, so quantizing fmlp_pack's output equals packing the
+ * quantized matrices: quantize packed_Wgu [2I x d] (K = d) and W_down
+ * [d x I] (K = I) for fmlp_forward_q8.
+ *
+ *   W      : bf16 [rows x K], K a multiple of 64
+ *   q      : int8 [rows x K], caller-allocated
+ *   scales : f32 [rows x K/64], caller-allocated
+ * Bit-exact: the same q and scales on every run.
+ */
+FMLP_API fmlp_status fmlp_quantize_q8(const void* W, int64_t rows, int64_t K, void* q,
+                                      float* scales, void* stream);
+
+/*
+ * fmlp_forward_q8 -- the MLP block (steps a1-a6) on int8 weights from
+ * fmlp_quantize_q8: fmlp_forward with W_gate, W_up and W_down replaced by
+ * their dequantized values q * s.  Decode batches only: 1 <= M <= 4 token
+ * rows, d and I multiples of 512, M*d*4 and M*I*4 bytes within shared
+ * memory (about 200 KB); other requests return FMLP_ERR_UNSUPPORTED.  About
+ * 1.06 bytes of weights per element are streamed instead of 2.
+ *
+ *   packed_q, packed_scales : fmlp_pack's [2I x d] matrix quantized (int8,
+ *                             f32 [2I x d/64]) with the same tile_T
+ *   W_down_q, W_down_scales : W_down [d x I] quantized (int8, f32 [d x I/64])
+ *   out                     : f32 [M x d], written by one thread per element
+ *                             (no atomics: the same bits on every run)
+ *   other arguments, workspace included, as in fmlp_forward.
+ * Two launches (gate-up GEMV with the SwiGLU epilogue, down GEMV with the
+ * residual) on the CUDA cores; a is rounded to bf16 in between, as in
+ * fmlp_forward.
+ */
+FMLP_API fmlp_status fmlp_forward_q8(const void* x, int64_t M, const void* gamma, float eps,
+                                     const void* packed_q, const float* packed_scales, int tile_T,
+                                     const void* W_down_q, const float* W_down_scales, int64_t d,
+                                     int64_t I, const void* residual, float* out, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * fmlp_sum_partials -- the reduction of a tensor-parallel MLP block:
  *     out = sum_r partials[r] (+ residual)
  * When the intermediate dimension I is split over n ranks (each rank holding

@@ -21,7 +21,7 @@ __all__ = [
     "fmlp_gate_up_swiglu", "fmlp_down_proj", "fmlp_device_status", "fmlp_status_string",
     "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "fmlp_set_wait_timeout_ns", "fmlp_set_fault_injection",
     "fmlp_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "fmlp_forward_bf16",
-    "fmlp_sum_partials",
+    "fmlp_sum_partials", "fmlp_quantize_q8", "fmlp_forward_q8", "Q8_GROUP",
 ]
 
 FMLP_OK, FMLP_ERR_INVALID_ARG, FMLP_ERR_UNSUPPORTED, FMLP_ERR_CUDA, FMLP_ERR_TIMEOUT = range(5)
@@ -46,6 +46,8 @@ _SIGNATURES = {
     "fmlp_forward_noalloc": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp]),
     "fmlp_forward_bf16": (_int, [_vp, _i64, _vp, _f32, _vp, _int, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
     "fmlp_sum_partials": (_int, [ctypes.POINTER(_vp), _int, _i64, _i64, _vp, _vp, _int, _vp]),
+    "fmlp_quantize_q8": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "fmlp_forward_q8": (_int, [_vp, _i64, _vp, _f32, _vp, _vp, _int, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -252,6 +254,50 @@ def fmlp_sum_partials(partials, out, residual=None, stream=None) -> None:
     _check_status(lib.fmlp_sum_partials(arr, len(partials), M, d, _ptr(residual), _ptr(out),
                                         int(out.dtype == torch.bfloat16), _stream(stream)),
                   "fmlp_sum_partials")
+
+
+Q8_GROUP = 64   # elements per scale of the int8 weight format (include/fmlp.h)
+
+
+def fmlp_quantize_q8(W, q, scales, stream=None) -> None:
+    """q int8 [rows x K], scales f32 [rows x K/64] <- the int8 format of W bf16 [rows x K]."""
+    _bf16(W, "W")
+    rows, K = _dims2(W, "W")
+    _check(W, "W", torch.bfloat16, (rows, K))
+    _check(q, "q", torch.int8, (rows, K))
+    _check(scales, "scales", torch.float32, (rows, K // Q8_GROUP))
+    _on_device(W=W, q=q, scales=scales)
+    _check_status(lib.fmlp_quantize_q8(_ptr(W), rows, K, _ptr(q), _ptr(scales), _stream(stream)),
+                  "fmlp_quantize_q8")
+
+
+def fmlp_forward_q8(x, gamma, eps: float, packed_q, packed_scales, tile_T: int, W_down_q,
+                    W_down_scales, out, workspace, residual=None, stream=None) -> None:
+    """out [M x d] (f32) <- the MLP block of x on int8 weights (fmlp_quantize_q8's)."""
+    _bf16(x, "x")
+    M, d = _dims2(x, "x")
+    d2, I = _dims2(W_down_q, "W_down_q")
+    if d2 != d:
+        raise ValueError(f"W_down_q has {d2} rows, x has {d} columns")
+    _check(x, "x", torch.bfloat16, (M, d))
+    _check(gamma, "gamma", torch.bfloat16, (d,))
+    _check(packed_q, "packed_q", torch.int8, (2 * I, d))
+    _check(packed_scales, "packed_scales", torch.float32, (2 * I, d // Q8_GROUP))
+    _check(W_down_q, "W_down_q", torch.int8, (d, I))
+    _check(W_down_scales, "W_down_scales", torch.float32, (d, I // Q8_GROUP))
+    _check(residual, "residual", torch.bfloat16, (M, d), optional=True)
+    _check(out, "out", torch.float32, (M, d))
+    _check_workspace(workspace, fmlp_workspace_bytes(M, d, I))
+    _on_device(x=x, gamma=gamma, packed_q=packed_q, packed_scales=packed_scales,
+               W_down_q=W_down_q, W_down_scales=W_down_scales, residual=residual, out=out,
+               workspace=workspace)
+    _check_status(lib.fmlp_forward_q8(_ptr(x), M, _ptr(gamma), eps, _ptr(packed_q),
+                                      _ptr(packed_scales), tile_T, _ptr(W_down_q),
+                                      _ptr(W_down_scales), d, I, _ptr(residual), _ptr(out),
+                                      _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(stream)),
+                  "fmlp_forward_q8")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20   # FMLP_NOALLOC_SCRATCH_BYTES in include/fmlp.h

@@ -158,6 +158,14 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Row of gate row i in the packed gate/up matrix (fmlp_pack): tile t of T
+// pairs holds gate rows iT..iT+T-1 and then their up rows, so the up row of i
+// is T rows further on.
+__device__ __forceinline__ int64_t gate_row(int i, int T) {
+  const int t = i / T;
+  return (int64_t)2 * T * t + (i - t * T);
+}
+
 // SiLU(g) * u in f32.  For g << 0, expf(-g) overflows to +inf and g/inf = -0.
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + expf(-g)) * u;

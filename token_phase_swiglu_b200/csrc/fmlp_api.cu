@@ -360,6 +360,45 @@ fmlp_status fmlp_forward_bf16(const void* x, int64_t M, const void* gamma, float
                       out, workspace, workspace_bytes, stream);
 }
 
+fmlp_status fmlp_quantize_q8(const void* W, int64_t rows, int64_t K, void* q, float* scales,
+                             void* stream) {
+  if (!W || !q || !scales || rows < 1 || K < 64 || K % 64 != 0 || K > kMaxI)
+    return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(q) || !aligned16(scales)) return FMLP_ERR_INVALID_ARG;
+  const DeviceInfo* dev = nullptr;
+  fmlp_status st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  cudaError_t e = launch_quantize_q8(W, rows, K, q, scales, *dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
+fmlp_status fmlp_forward_q8(const void* x, int64_t M, const void* gamma, float eps,
+                            const void* packed_q, const float* packed_scales, int tile_T,
+                            const void* W_down_q, const float* W_down_scales, int64_t d,
+                            int64_t I, const void* residual, float* out, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  fmlp_status st = check_common(M, d, I, workspace, workspace_bytes);
+  if (st != FMLP_OK) return st;
+  if (!gamma || !packed_q || !packed_scales || !W_down_q || !W_down_scales)
+    return FMLP_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !out)) return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(packed_q) || !aligned16(packed_scales) ||
+      !aligned16(W_down_q) || !aligned16(W_down_scales) || !aligned16(out) ||
+      !aligned16(residual))
+    return FMLP_ERR_INVALID_ARG;
+  if (!eps_ok(eps) || !tile_ok(tile_T, I)) return FMLP_ERR_INVALID_ARG;
+  if (M == 0) return FMLP_OK;
+  const DeviceInfo* dev = nullptr;
+  st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  if (!q8_supported(M, d, I, tile_T, *dev)) return FMLP_ERR_UNSUPPORTED;
+  void* a = (char*)workspace + workspace_layout(M, d, I).a;
+  cudaError_t e = launch_forward_q8(x, M, gamma, eps, packed_q, packed_scales, tile_T, W_down_q,
+                                    W_down_scales, d, I, residual, out, nullptr, a,
+                                    (uint32_t*)workspace, *dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
 fmlp_status fmlp_sum_partials(const float* const* partials, int n, int64_t M, int64_t d,
                               const void* residual, void* out, int out_bf16, void* stream) {
   if (n < 1 || n > kMaxPartials || M < 0 || d <= 0 || d % 8 != 0 || d > kMaxD)

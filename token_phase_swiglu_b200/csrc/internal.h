@@ -136,6 +136,16 @@ cudaError_t launch_sum_partials(const float* const* parts, int n, int64_t M, int
                                 const void* residual, float* out_f32, void* out_bf16,
                                 const DeviceInfo& dev, cudaStream_t stream);
 
+// int8 weights (csrc/q8.cu): groups of 64 along K with one f32 scale each.
+bool q8_supported(int64_t M, int64_t d, int64_t I, int T, const DeviceInfo& dev);
+cudaError_t launch_quantize_q8(const void* W, int64_t rows, int64_t K, void* q, float* s,
+                               const DeviceInfo& dev, cudaStream_t stream);
+cudaError_t launch_forward_q8(const void* x, int64_t M, const void* gamma, float eps,
+                              const void* Pq, const float* Ps, int T, const void* Wdq,
+                              const float* Wds, int64_t d, int64_t I, const void* residual,
+                              float* out, void* out_bf16, void* a, uint32_t* status,
+                              const DeviceInfo& dev, cudaStream_t stream);
+
 // out = residual or zero (for a down GEMM with no gate-up prologue before it).
 cudaError_t launch_out_init(float* out, const void* residual, int64_t M, int64_t d,
                             const DeviceInfo& dev, cudaStream_t stream);
