@@ -79,7 +79,8 @@ def measured_peaks() -> dict:
 # the source files each kernel is built from (its traffic record goes stale
 # when any of them changes)
 KERNEL_SOURCES = {
-    "fused_decode": ["stream.cu", "common.cuh", "internal.h"],
+    "fused_decode": ["stream.cu", "ring.cuh", "common.cuh", "internal.h"],
+    "q8_stream": ["q8.cu", "ring.cuh", "common.cuh", "internal.h"],
     "tc_gemm": ["tc.cu", "tcgen05.cuh", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
     "tc_layer": ["layer.cu", "tcgen05.cuh", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
 }
@@ -555,7 +556,7 @@ def roofline_entry(run: WorkloadRun, ms_step: float, gu_ms, sustained: bool = Fa
     single = run.per_step is not None and run.per_step == L
     if run.quant:
         # the int8 path: two launches per layer, both weight streams
-        kname, kms = "q8_gateup + q8_down", ms_step / L
+        kname, kms = "q8_stream", ms_step / L
         timing = "timed region / layers (two launches per layer, back to back in a CUDA graph)"
         kbytes, kflops = q8_bytes(M, d, I), 6 * M * d * I
     elif single:
@@ -572,9 +573,10 @@ def roofline_entry(run: WorkloadRun, ms_step: float, gu_ms, sustained: bool = Fa
     else:
         bound, kpeak, src, unit, work = "hbm", peak, peak_src, "GB/s", kbytes
     achieved = work / (kms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
-    traffic = None if run.quant else recorded_traffic(
-        "fused_decode" if kname == "fused_decode" else
-        ("tc_layer" if kname == "tc_layer" else "tc_gemm"), w.name)
+    # DRAM bytes of one layer (the two int8 launches summed) or of the gate-up launch
+    traffic = recorded_traffic(
+        kname if kname in ("fused_decode", "tc_layer", "q8_stream") else "tc_gemm",
+        w.name + ("_q8" if run.quant else ""))
     return {"bound": bound, "kernel": kname, "achieved": round(achieved, 2), "peak": kpeak,
             "peak_source": src, "unit": unit, "frac": round(achieved / kpeak, 4),
             "traffic": traffic, "algorithmic_per_launch": work, "avg_launch_ms": round(kms, 5),

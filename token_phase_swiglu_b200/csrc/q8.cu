@@ -16,8 +16,9 @@
 // streaming kernels: one CTA per SM, whose producer lane streams groups of
 // whole rows (int8 values, then their scales) into a ring of shared-memory
 // stages with bulk copies, and 16 consumer warps that share every stage --
-// warp c takes row c % R of the stage's R rows and column part c / R -- and
-// leave their warp-reduced sums in shared memory, so no consumer waits for
+// each takes a few of the stage's rows over one column part, so that one
+// activation load serves several rows -- and leave their warp-reduced sums
+// in shared memory, so no consumer waits for
 // another until the phase ends; then each row's parts are summed in a fixed
 // order (the result does not depend on timing).  The activations sit in
 // shared memory as f32 in a chunk-interleaved order -- element e of 16-byte
@@ -39,7 +40,7 @@ constexpr int kQ8Group = 64;                         // elements per scale
 constexpr int kQ8Consumers = 16;                     // consumer warps
 constexpr int kQ8Threads = (kQ8Consumers + 1) * 32;  // warp 0 produces
 constexpr int kQ8BarConsumers = 1;                   // named barrier: consumer-only sync
-constexpr size_t kQ8MaxStageBytes = 64 * 1024;
+constexpr size_t kQ8MaxStageBytes = 72 * 1024;  // 16 rows of 4096 with their scales
 constexpr int kQ8StaticSlack = 2048;                 // static shared memory of the kernels and slack
 
 // Index of element k in the chunk-interleaved activation layout.
@@ -131,6 +132,7 @@ struct Q8Params {
   int M, d, I, T;
   int K;                    // row length: d (gate-up) or I (down)
   int R;                    // rows per stage: gate-up G gate rows then their G up rows (R = 2G)
+  int rw;                   // rows of a stage per consumer warp (divides R, <= q8_rows_per_warp)
   int groups;               // stages in the phase: I / G (gate-up) or d / R (down)
   int stages, stage_bytes;
 };
@@ -139,9 +141,7 @@ struct Q8Params {
 __host__ __device__ constexpr size_t q8_stage_bytes(int R, int K) {
   return align128((size_t)R * K + (size_t)R * (K / kQ8Group) * sizeof(float));
 }
-__host__ __device__ constexpr size_t q8_part_bytes(int max_groups, int mt) {
-  return align128((size_t)max_groups * kQ8Consumers * mt * sizeof(float));
-}
+
 
 template <bool GATE>
 __device__ void q8_produce(Producer& pr, const Q8Params& p, int g0, int ng) {
@@ -170,49 +170,117 @@ __device__ void q8_produce(Producer& pr, const Q8Params& p, int g0, int ng) {
   }
 }
 
-// Consumer warp c: row c % R of every stage, chunks [c0, c1) of that row
-// (part c / R of R's kQ8Consumers / R parts).  Leaves each stage's sums in
+// Rows of a stage that one consumer warp takes at the same columns: each
+// activation load from shared memory then serves that many rows (2 for 3-4
+// token rows, whose activations and accumulators take more registers).
+template <int MT>
+__host__ __device__ constexpr int q8_rows_per_warp() { return MT <= 2 ? 4 : 2; }
+static_assert(q8_rows_per_warp<1>() == 4 && q8_rows_per_warp<3>() == 2, "q8_part_bytes agrees");
+
+// Column parts per row of a stage of R rows: the kQ8Consumers warps take rw
+// rows each, so R / rw warps span the rows once and each row is split
+// kQ8Consumers rw / R ways.
+__host__ __device__ constexpr int q8_parts(int R, int rw) { return kQ8Consumers * rw / R; }
+// Bytes of the consumers' sums per CTA: every warp leaves rw <= RW row sums
+// per token row per stage.
+__host__ __device__ constexpr size_t q8_part_bytes(int max_groups, int mt) {
+  return align128((size_t)max_groups * kQ8Consumers * (mt <= 2 ? 4 : 2) * mt * sizeof(float));
+}
+
+// Consumer warp c takes rows [r0, r0 + rw) of every stage (rw <= RW),
+// r0 = rw (c % (R / rw)), and chunks [c0, c1) of them: part c / (R / rw) of
+// the rows' kQ8Consumers rw / R column parts.  Leaves each stage's sums in
 // part[((j R + r) parts + part) MT + m].
 template <int MT>
 __device__ bool q8_consume(Consumer& cs, const Q8Params& p, int ng, const float* act,
                            float* part) {
+  constexpr int RW = q8_rows_per_warp<MT>();
   const int c = (threadIdx.x >> 5) - 1, lane = cs.lane;
-  const int R = p.R, parts = kQ8Consumers / R, r = c % R, pt = c / R;
+  const int R = p.R, rw = p.rw, groups_r = R / rw, parts = q8_parts(R, rw);
+  const int r0 = rw * (c % groups_r), pt = c / groups_r;
   const int K = p.K, nc = K / 16, gpr = K / kQ8Group;
   const int c0 = pt * nc / parts, c1 = (pt + 1) * nc / parts;
   for (int j = 0; j < ng; ++j) {
     const uint8_t* buf = cs.wait_full();
     if (!buf) return false;
-    const uint8_t* wrow = buf + (size_t)r * K;
-    const float* srow = reinterpret_cast<const float*>(buf + (size_t)R * K) + r * gpr;
-    uint64_t acc[MT];
+    const uint8_t* wrow = buf + (size_t)r0 * K;
+    const float* srow = reinterpret_cast<const float*>(buf + (size_t)R * K) + r0 * gpr;
+    uint64_t acc[RW][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0ull;
+    for (int rr = 0; rr < RW; ++rr)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[rr][m] = 0ull;
     for (int ch = c0 + lane; ch < c1; ch += 32) {
-      const uint4 qv = lds128(wrow + 16 * ch);
-      const float sc = srow[ch >> 2];
-      uint64_t w[8];
-      dequant16(qv, w);
       const float* ab = act + ((ch >> 5) << 9) + ((ch & 31) << 2);
+      if constexpr (MT <= 2) {
+        // activations of every token row first, then one row's weights at a time
+        float4 a4[MT][4];
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const float* am = ab + m * K;
-        uint64_t t = 0ull;
+        for (int m = 0; m < MT; ++m)
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const float4 a4 = *reinterpret_cast<const float4*>(am + (jj << 7));
-          t = ffma2(w[2 * jj], pk2(a4.x, a4.y), t);
-          t = ffma2(w[2 * jj + 1], pk2(a4.z, a4.w), t);
+          for (int jj = 0; jj < 4; ++jj)
+            a4[m][jj] = *reinterpret_cast<const float4*>(ab + m * K + (jj << 7));
+#pragma unroll
+        for (int rr = 0; rr < RW; ++rr) {
+          if (rr < rw) {
+            uint64_t w[8];
+            dequant16(lds128(wrow + (size_t)rr * K + 16 * ch), w);
+            const float sc = srow[rr * gpr + (ch >> 2)];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              uint64_t t = 0ull;
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                t = ffma2(w[2 * jj], pk2(a4[m][jj].x, a4[m][jj].y), t);
+                t = ffma2(w[2 * jj + 1], pk2(a4[m][jj].z, a4[m][jj].w), t);
+              }
+              acc[rr][m] = ffma2(t, pk2(sc, sc), acc[rr][m]);
+            }
+          }
         }
-        acc[m] = ffma2(t, pk2(sc, sc), acc[m]);
+      } else {
+        // the rows' weights first, then one token row's activations at a time
+        uint64_t w[RW][8];
+        float sc[RW];
+#pragma unroll
+        for (int rr = 0; rr < RW; ++rr) {
+          if (rr < rw) {
+            dequant16(lds128(wrow + (size_t)rr * K + 16 * ch), w[rr]);
+            sc[rr] = srow[rr * gpr + (ch >> 2)];
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          float4 a4[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            a4[jj] = *reinterpret_cast<const float4*>(ab + m * K + (jj << 7));
+#pragma unroll
+          for (int rr = 0; rr < RW; ++rr) {
+            if (rr < rw) {
+              uint64_t t = 0ull;
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                t = ffma2(w[rr][2 * jj], pk2(a4[jj].x, a4[jj].y), t);
+                t = ffma2(w[rr][2 * jj + 1], pk2(a4[jj].z, a4[jj].w), t);
+              }
+              acc[rr][m] = ffma2(t, pk2(sc[rr], sc[rr]), acc[rr][m]);
+            }
+          }
+        }
       }
     }
     cs.release();
-    float* dst = part + ((j * R + r) * parts + pt) * MT;
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      const float v = warp_sum(hsum2(acc[m]));
-      if (lane == 0) dst[m] = v;
+    for (int rr = 0; rr < RW; ++rr) {
+      if (rr < rw) {
+        float* dst = part + ((j * R + r0 + rr) * parts + pt) * MT;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float v = warp_sum(hsum2(acc[rr][m]));
+          if (lane == 0) dst[m] = v;
+        }
+      }
     }
   }
   return true;
@@ -260,20 +328,34 @@ __device__ void q8_stage_x(const Q8Params& p, int mt, float* act, float (*red)[M
   }
 }
 
-// a (bf16) as f32 into the interleaved layout, rows >= mt zero.  Consumer threads.
+// a (bf16) as f32 into the interleaved layout, rows >= mt zero.  Consumer
+// threads; each issues the loads of several vectors before storing any.
 template <int MT>
 __device__ void q8_stage_a(const Q8Params& p, int mt, float* act) {
-  const int I = p.I, ct = threadIdx.x - 32;
-  for (int v = ct; v < I / 8; v += kQ8Consumers * 32) {
+  constexpr int V = MT <= 2 ? 4 : 2;
+  const int I = p.I, ct = threadIdx.x - 32, nv = I / 8;
+  for (int v0 = ct; v0 < nv; v0 += V * kQ8Consumers * 32) {
+    uint4 av[V][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      uint4 av = make_uint4(0, 0, 0, 0);
-      if (m < mt) av = ld_keep(p.a + (int64_t)m * I + (int64_t)v * 8);
-      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+    for (int u = 0; u < V; ++u)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        act[m * I + act_index(v * 8 + 2 * e)] = bf16lo(aw[e]);
-        act[m * I + act_index(v * 8 + 2 * e + 1)] = bf16hi(aw[e]);
+      for (int m = 0; m < MT; ++m) {
+        const int v = v0 + u * kQ8Consumers * 32;
+        av[u][m] = make_uint4(0, 0, 0, 0);
+        if (v < nv && m < mt) av[u][m] = ld_keep(p.a + (int64_t)m * I + (int64_t)v * 8);
+      }
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      const int v = v0 + u * kQ8Consumers * 32;
+      if (v >= nv) break;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint32_t aw[4] = {av[u][m].x, av[u][m].y, av[u][m].z, av[u][m].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          act[m * I + act_index(v * 8 + 2 * e)] = bf16lo(aw[e]);
+          act[m * I + act_index(v * 8 + 2 * e + 1)] = bf16hi(aw[e]);
+        }
       }
     }
   }
@@ -322,7 +404,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_stream(const __grid_constant
       q8_stage_x<MT>(p, mt, act, red, rinv);
       const bool ok = q8_consume<MT>(cs, p, ng, act, part);
       if (!consumer_barrier_any<kQ8Consumers * 32>(kQ8BarConsumers, !ok)) {
-        const int G = p.R / 2, parts = kQ8Consumers / p.R;
+        const int G = p.R / 2, parts = q8_parts(p.R, p.rw);
         for (int i = ct; i < ng * G; i += kQ8Consumers * 32) {
           const int j = i / G, gp = i - j * G;
           const float* pg = part + ((j * p.R + gp) * parts) * MT;
@@ -344,7 +426,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_stream(const __grid_constant
       q8_stage_a<MT>(p, mt, act);
       const bool ok = q8_consume<MT>(cs, p, ng, act, part);
       if (!consumer_barrier_any<kQ8Consumers * 32>(kQ8BarConsumers, !ok)) {
-        const int parts = kQ8Consumers / p.R;
+        const int parts = q8_parts(p.R, p.rw);
         for (int i = ct; i < ng * p.R; i += kQ8Consumers * 32) {
           const int64_t n = (int64_t)g0 * p.R + i;
           const float* pr = part + (i * parts) * MT;
@@ -369,13 +451,34 @@ __global__ void __launch_bounds__(kQ8Threads, 1) q8_stream(const __grid_constant
 // host side
 // ---------------------------------------------------------------------------
 struct Q8Plan {
-  int R = 0, stages = 0, groups = 0;
+  int R = 0, rw = 0, stages = 0, groups = 0;
   size_t stage_bytes = 0, smem = 0;
 };
 
+// Rows of a stage per consumer warp: the largest rw <= rw_max (each
+// activation load then serves rw rows) among those that keep the most lanes
+// busy -- a row of nc 16-byte chunks is split into 16 rw / R parts, one
+// chunk per lane at a time, so a part of 48 chunks leaves a quarter of the
+// lanes idle on its second pass.
+int q8_choose_rw(int R, int nc, int rw_max) {
+  int best = 1;
+  double best_eff = -1.0;
+  for (int rw = std::min(rw_max, R); rw >= 1; rw /= 2) {
+    const int parts = q8_parts(R, rw);
+    const int longest = (nc + parts - 1) / parts;
+    const double eff = (double)nc / parts / (32.0 * ((longest + 31) / 32));
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = rw;
+    }
+  }
+  return best;
+}
+
 // Rows per stage and ring depth for one phase: the largest stage (at most
-// 64 KB, fewer copies per byte) that leaves a ring of at least three stages
-// beside the activations and the consumers' sums.
+// 72 KB; the number of copies, more than their bytes, limits a bulk-copy
+// ring) that leaves a ring of at least three stages beside the activations
+// and the consumers' sums.
 Q8Plan q8_plan(int64_t M, int64_t d, int64_t I, int T, bool gate, const DeviceInfo& dev) {
   const size_t budget = (size_t)dev.max_smem_optin - kQ8StaticSlack;
   const int K = (int)(gate ? d : I);
@@ -395,6 +498,7 @@ Q8Plan q8_plan(int64_t M, int64_t d, int64_t I, int T, bool gate, const DeviceIn
     if (fit < 3) continue;
     pl.stages = (int)std::min<size_t>(kMaxStages, fit);
     pl.smem = fixed + (size_t)pl.stages * pl.stage_bytes;
+    pl.rw = q8_choose_rw(R, K / 16, M <= 2 ? 4 : 2);
     return pl;
   }
   return Q8Plan();
@@ -420,6 +524,7 @@ cudaError_t launch_phase(Q8Params p, const Q8Plan& pl, const DeviceInfo& dev,
   cudaError_t e = allow_q8_smem(k, dev);
   if (e != cudaSuccess) return e;
   p.R = pl.R;
+  p.rw = pl.rw;
   p.groups = pl.groups;
   p.stages = pl.stages;
   p.stage_bytes = (int)pl.stage_bytes;
