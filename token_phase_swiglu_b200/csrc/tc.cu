@@ -56,9 +56,11 @@ enum Epi { kEpiSwiGLU = 0, kEpiDown = 1 };
 // ---------------------------------------------------------------------------
 // Segment s of this CTA's work: tile t, stages [kb0, kb1).  Segments
 // 0..dp-1 are the whole tiles of the data-parallel rounds; then the
-// stream-K range [u0, u1).  Returns false past the end.
+// stream-K range [u0, u1).  With a split schedule, segment s is item
+// s * ctas + this CTA.  Returns false past the end.
 __device__ __forceinline__ bool segment(const Sched& S, int64_t u0, int64_t u1, int s, int& t,
                                         int& kb0, int& kb1) {
+  if (S.split) return s < S.dp && S.split_item(s * S.ctas + (int)blockIdx.x, t, kb0, kb1);
   if (s < S.dp) {
     t = s * S.ctas + (int)blockIdx.x;
     kb0 = 0;
@@ -581,6 +583,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 // Segment s of stream-K/data-parallel work unit `me` (a CTA, or a CTA pair).
 __device__ __forceinline__ bool segment_of(const Sched& S, int me, int64_t u0, int64_t u1, int s,
                                            int& t, int& kb0, int& kb1) {
+  if (S.split) return s < S.dp && S.split_item(s * S.ctas + me, t, kb0, kb1);
   if (s < S.dp) {
     t = s * S.ctas + me;
     kb0 = 0;
@@ -1189,6 +1192,26 @@ void fill_common(TcParams& p, const TcPlan& pl, int epi, int64_t M, int rows, in
   // a stream-K tile has only a few contributors.
   const int waves = p.sched.tiles / p.sched.ctas, rest = p.sched.tiles % p.sched.ctas;
   p.sched.dp = pl.ntok == 1 ? 0 : (2 * rest >= p.sched.ctas ? waves : std::max(0, waves - 1));
+  p.sched.split = 0;
+  if (epi == kEpiDown && pl.ntok > 1) {
+    // The down GEMM adds every share into out, so it can run all of its work
+    // as data-parallel (tile, k-part) items: the CTAs of a round then share
+    // each weight stage across the token tiles, where a stream-K remainder
+    // read a weight tile once per token tile (8B prefill: 598 MB of DRAM
+    // reads against 176 MB).  The k-part count fills the rounds best.
+    const int max_split = std::max(1, std::min(8, p.sched.KB / 4));
+    double best = -1.0;
+    for (int sp = 1; sp <= max_split; ++sp) {
+      const int64_t items = (int64_t)p.sched.tiles * sp;
+      const int64_t rounds = (items + p.sched.ctas - 1) / p.sched.ctas;
+      const double eff = (double)items / (double)(rounds * p.sched.ctas);
+      if (eff > best + 1e-3) {
+        best = eff;
+        p.sched.split = sp;
+        p.sched.dp = (int)rounds;
+      }
+    }
+  }
   p.partials = ws.partials;
   p.counters = ws.counters;
   p.status = ws.status;

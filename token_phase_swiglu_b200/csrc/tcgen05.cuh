@@ -129,9 +129,25 @@ struct Sched {
   int tiles;   // row tiles x token tiles
   int ntok;    // token tiles (tile index = row_tile * ntok + token_tile)
   int ctas;    // grid size
-  int dp;      // data-parallel rounds (whole tiles per CTA)
+  int dp;      // data-parallel rounds (whole tiles per CTA, or split items)
+  int split = 0;  // > 0: every round is data-parallel over (tile, k-part) items, `split`
+                  // k-parts per tile, ordered so that a round's items share weight k-parts
+                  // (down GEMM only: its shares are added into out); no stream-K part
   __device__ __forceinline__ int sk_tile0() const { return dp * ctas; }
-  __device__ __forceinline__ int64_t units() const { return (int64_t)(tiles - sk_tile0()) * KB; }
+  __device__ __forceinline__ int64_t units() const {
+    return split ? 0 : (int64_t)(tiles - sk_tile0()) * KB;
+  }
+  // Item i of the split schedule: tile t, stages [kb0, kb1).  Items run in
+  // the order (row tile, k-part, token tile), so the CTAs of one round that
+  // take the token tiles of a row tile read the same weight stages together.
+  __device__ __forceinline__ bool split_item(int i, int& t, int& kb0, int& kb1) const {
+    if (i >= tiles * split) return false;
+    const int tt = i % ntok, rest = i / ntok, kp = rest % split, rt = rest / split;
+    t = rt * ntok + tt;
+    kb0 = (int)((int64_t)KB * kp / split);
+    kb1 = (int)((int64_t)KB * (kp + 1) / split);
+    return true;
+  }
   // stream-K unit range of CTA c (units counted from the first stream-K tile)
   __device__ __forceinline__ void range(int c, int64_t& u0, int64_t& u1) const {
     const int64_t U = units(), per = U / ctas, rem = U % ctas;
