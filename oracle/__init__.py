@@ -25,6 +25,10 @@ and the gate/up interleave, a pure permutation of rows at tile granularity.
 ``quant.py`` restates this build's int8 weight format (the pages name
 quantized weight streaming but give no format) and the block on it.
 
+``attn.py`` restates the token-phase attention step of the same pages
+(section 三, components 1-2 and Figure 3: GKVC's in-place KV append at the
+Eq(2) address, TPSFLAT's RoPE + QK^T + Softmax + PV).
+
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, exact invariants, brute force on tiny shapes and the page-described
 row order -- never against the CUDA path.  No function here is "parity
@@ -51,4 +55,12 @@ from .quant import (  # noqa: F401
     quantize_rows,
     dequantize_rows,
     fused_mlp_q8,
+)
+from .attn import (  # noqa: F401
+    gkvc_step,
+    rope_angles,
+    rope,
+    decode_attention,
+    kv_append,
+    token_attention,
 )

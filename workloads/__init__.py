@@ -18,6 +18,12 @@ problem with seed ``s`` is split into fixed chunks of 2**22 values; chunk
 the bytes do not depend on how many threads fill them.
 
 No trained weights are used: the model names in WORKLOADS only give shapes.
+
+The token-phase attention workloads (ATTN_WORKLOADS) draw, from tensor ids of
+their own: the new token's q [B x H x D], k and v [B x H_kv x D], and the
+KV-cache regions [B x H_kv x N_max x D] that earlier tokens filled, all
+N(0, 1) in bf16 (unit-variance projections, so scores q.k/sqrt(D) are of
+order one); every sequence's new token sits at position n_ctx - 1.
 """
 
 from __future__ import annotations
@@ -33,6 +39,7 @@ CHUNK = 1 << 22
 
 # tensor ids inside one problem's seed space
 TID_X, TID_GAMMA, TID_WGATE, TID_WUP, TID_WDOWN, TID_RESID = 0, 1, 2, 3, 4, 5
+TID_Q, TID_KNEW, TID_VNEW, TID_KCACHE, TID_VCACHE = 6, 7, 8, 9, 10
 
 
 @dataclass(frozen=True)
@@ -135,3 +142,43 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """The raw bf16 bit patterns of a host tensor, as uint16 (a view, no arithmetic)."""
     assert t.dtype == torch.bfloat16
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclass(frozen=True)
+class AttnWorkload:
+    name: str
+    B: int          # sequences, one new token each
+    H: int          # query heads
+    H_kv: int       # KV heads (H / H_kv queries share one)
+    D: int          # head dimension
+    n_ctx: int      # rows held after the step (the new token is row n_ctx - 1)
+    n_max: int      # rows of each head's cache region (N_p + N_r)
+    theta: float    # RoPE base
+    layers: int = 1  # independent layers (own caches each)
+
+    @property
+    def kv_bytes(self) -> int:
+        """K and V rows the step reads (bf16), the new row included."""
+        return 2 * self.B * self.H_kv * self.n_ctx * self.D * 2
+
+
+# Shapes of the attention side of the same models: Phi-3-mini-4k (32 heads of
+# 96, no grouping, a full 4k context) and Llama-3.1-8B (32 query heads over 8
+# KV heads of 128) with eight 4k sequences in flight.
+ATTN_WORKLOADS = {
+    "attn_tiny": AttnWorkload("attn_tiny", 2, 4, 2, 64, 300, 320, 10000.0),
+    "phi3_attn": AttnWorkload("phi3_attn", 1, 32, 32, 96, 4096, 4096, 10000.0, layers=32),
+    "llama8b_attn": AttnWorkload("llama8b_attn", 8, 32, 8, 128, 4096, 4096, 500000.0, layers=8),
+}
+
+
+def make_attn_problem(B: int, H: int, H_kv: int, D: int, n_max: int, seed: int = 0) -> dict:
+    """q, k_new, v_new and the two cache regions of one attention step (bf16, host)."""
+    return {
+        "q": normal_bf16(seed, TID_Q, (B, H, D)),
+        "k_new": normal_bf16(seed, TID_KNEW, (B, H_kv, D)),
+        "v_new": normal_bf16(seed, TID_VNEW, (B, H_kv, D)),
+        "k_cache": normal_bf16(seed, TID_KCACHE, (B, H_kv, n_max, D)),
+        "v_cache": normal_bf16(seed, TID_VCACHE, (B, H_kv, n_max, D)),
+    }
+
