@@ -264,10 +264,62 @@ FMLP_API fmlp_status fmlp_sum_partials(const float* const* partials, int n, int6
                                        void* stream);
 
 /*
+ * Token-phase attention step: the GKVC and TPSFLAT components of "FastTPS:
+ * An Optimized Method for LLM Token Phase for AI Accelerators" (xllm-io
+ * paper review), section 三, components 1-2, Figure 3 and Eq(2).
+ *
+ * fmlp_attn_workspace_bytes -- bytes of the workspace fmlp_attn_decode needs
+ * for B sequences of H query heads over H_kv KV heads of dimension D (0 if
+ * the shape is not taken).  Zero-fill it once; the calls keep it zero.
+ */
+FMLP_API size_t fmlp_attn_workspace_bytes(int64_t B, int H, int H_kv, int D);
+
+/*
+ * fmlp_attn_decode -- one new token per sequence: RoPE on q and k at the
+ * token's position, in-place append of the new K and V rows to the cache,
+ * and the attention of every query head over the cache rows 0..pos.
+ *
+ *   q        : bf16 [B x H x D], the new token's queries (before RoPE)
+ *   k_new    : bf16 [B x H_kv x D], its keys (before RoPE)
+ *   v_new    : bf16 [B x H_kv x D], its values
+ *   k_cache,
+ *   v_cache  : bf16 [B x H_kv x n_max x D], head-major regions of n_max rows
+ *              (N_p + N_r of Eq(2)); rows 0..pos[b]-1 hold the earlier tokens.
+ *              The call writes row pos[b] of every KV head of sequence b --
+ *              the rotated key rounded to bf16 (nearest even), and v_new --
+ *              at the Eq(2) offset ((b H_kv + g) n_max + pos[b]) D, and reads
+ *              nothing past it.
+ *   pos      : int32 [B] on the device, the new token's position (rows held);
+ *              0 <= pos[b] < n_ctx <= n_max.  A position outside that range is
+ *              not processed: its sequence's outputs and cache are left as
+ *              they were and fmlp_device_status reports FMLP_ERR_INVALID_ARG.
+ *   n_ctx    : host-side bound on every pos[b] + 1; the work is split over
+ *              n_ctx rows per sequence, so a tight bound balances best.
+ *   theta    : RoPE base (> 0): angle_i = pos * theta^(-2i/D), pairs (i, i + D/2)
+ *   out      : f32 [B x H x D]: o_h = softmax(q'_h . K_g / sqrt(D)) V_g with
+ *              g = h / (H / H_kv), accumulated in f32
+ *   workspace: fmlp_attn_workspace_bytes(B, H, H_kv, D) bytes, 16-byte
+ *              aligned, zero-filled before first use.  After a call that
+ *              reported FMLP_ERR_TIMEOUT or FMLP_ERR_INVALID_ARG through
+ *              fmlp_device_status, zero it again before reuse.
+ * Shapes taken: D in {64, 96, 128}; H / H_kv in {1, 2, 4, 8}; B * H_kv * n_max
+ * < 2^31.  All pointers 16-byte aligned (pos 4-byte).  Runs after the
+ * previous work on `stream` (which may have written the cache or pos).
+ * Returns FMLP_ERR_INVALID_ARG before launching anything if an argument is
+ * outside these limits.
+ */
+FMLP_API fmlp_status fmlp_attn_decode(const void* q, const void* k_new, const void* v_new,
+                                      void* k_cache, void* v_cache, const int32_t* pos,
+                                      int64_t B, int H, int H_kv, int D, int64_t n_max,
+                                      int64_t n_ctx, float theta, float* out, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/*
  * fmlp_device_status -- synchronise `stream`, read the device status word in
  * `workspace` and reset it to zero.  Returns FMLP_ERR_TIMEOUT if a kernel
- * gave up a bounded wait since the last check, FMLP_OK otherwise (or
- * FMLP_ERR_CUDA / FMLP_ERR_INVALID_ARG).  After a timeout it also resets the
+ * gave up a bounded wait since the last check, FMLP_ERR_INVALID_ARG if a
+ * kernel met a device-side input out of range (an attention position),
+ * FMLP_OK otherwise (or FMLP_ERR_CUDA / FMLP_ERR_INVALID_ARG for the call).  After a timeout it also resets the
  * workspace's other control words, so the workspace can be used again; no
  * other call may be using the workspace meanwhile.
  */

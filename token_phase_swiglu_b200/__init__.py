@@ -22,6 +22,7 @@ __all__ = [
     "fmlp_last_cuda_error", "fmlp_kernel_launch_count", "fmlp_set_wait_timeout_ns", "fmlp_set_fault_injection",
     "fmlp_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "fmlp_forward_bf16",
     "fmlp_sum_partials", "fmlp_quantize_q8", "fmlp_forward_q8", "Q8_GROUP",
+    "fmlp_attn_workspace_bytes", "fmlp_attn_decode",
 ]
 
 FMLP_OK, FMLP_ERR_INVALID_ARG, FMLP_ERR_UNSUPPORTED, FMLP_ERR_CUDA, FMLP_ERR_TIMEOUT = range(5)
@@ -48,6 +49,9 @@ _SIGNATURES = {
     "fmlp_sum_partials": (_int, [ctypes.POINTER(_vp), _int, _i64, _i64, _vp, _vp, _int, _vp]),
     "fmlp_quantize_q8": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "fmlp_forward_q8": (_int, [_vp, _i64, _vp, _f32, _vp, _vp, _int, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "fmlp_attn_workspace_bytes": (_sz, [_i64, _int, _int, _int]),
+    "fmlp_attn_decode": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _i64, _i64, _f32,
+                                _vp, _vp, _sz, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -298,6 +302,40 @@ def fmlp_forward_q8(x, gamma, eps: float, packed_q, packed_scales, tile_T: int, 
                                       workspace.numel() * workspace.element_size(),
                                       _stream(stream)),
                   "fmlp_forward_q8")
+
+
+def fmlp_attn_workspace_bytes(B: int, H: int, H_kv: int, D: int) -> int:
+    n = lib.fmlp_attn_workspace_bytes(B, H, H_kv, D)
+    if n == 0:
+        raise FmlpError(FMLP_ERR_INVALID_ARG, "fmlp_attn_workspace_bytes: shape not taken")
+    return n
+
+
+def fmlp_attn_decode(q, k_new, v_new, k_cache, v_cache, pos, n_ctx: int, theta: float, out,
+                     workspace, stream=None) -> None:
+    """One token-phase attention step (RoPE, in-place KV append, attention over
+    the cache rows 0..pos); see include/fmlp.h for the layouts."""
+    _bf16(q, "q")
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [B, H, D] and the caches [B, H_kv, n_max, D]")
+    B, H, D = q.shape
+    H_kv, n_max = k_cache.shape[1], k_cache.shape[2]
+    _check(q, "q", torch.bfloat16, (B, H, D))
+    _check(k_new, "k_new", torch.bfloat16, (B, H_kv, D))
+    _check(v_new, "v_new", torch.bfloat16, (B, H_kv, D))
+    _check(k_cache, "k_cache", torch.bfloat16, (B, H_kv, n_max, D))
+    _check(v_cache, "v_cache", torch.bfloat16, (B, H_kv, n_max, D))
+    _check(pos, "pos", torch.int32, (B,))
+    _check(out, "out", torch.float32, (B, H, D))
+    _check_workspace(workspace, fmlp_attn_workspace_bytes(B, H, H_kv, D))
+    _on_device(q=q, k_new=k_new, v_new=v_new, k_cache=k_cache, v_cache=v_cache, pos=pos, out=out,
+               workspace=workspace)
+    _check_status(lib.fmlp_attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                       _ptr(v_cache), _ptr(pos), B, H, H_kv, D, n_max, n_ctx,
+                                       theta, _ptr(out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)),
+                  "fmlp_attn_decode")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20   # FMLP_NOALLOC_SCRATCH_BYTES in include/fmlp.h

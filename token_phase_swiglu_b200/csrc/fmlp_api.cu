@@ -24,6 +24,7 @@ cudaError_t g_info_err[kMaxDevices];
 
 constexpr int64_t kMaxD = 32768;
 constexpr int64_t kMaxI = 65536;
+constexpr int64_t kMaxAttnBatch = 65536;  // sequences per attention call
 
 inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }  // NULL passes
@@ -421,6 +422,34 @@ fmlp_status fmlp_sum_partials(const float* const* partials, int n, int64_t M, in
   return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
 }
 
+size_t fmlp_attn_workspace_bytes(int64_t B, int H, int H_kv, int D) {
+  if (B < 1 || B > kMaxAttnBatch || !attn_shape_ok(H, H_kv, D)) return 0;
+  return attn_layout(B, H, H_kv, D).total;
+}
+
+fmlp_status fmlp_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                             void* v_cache, const int32_t* pos, int64_t B, int H, int H_kv, int D,
+                             int64_t n_max, int64_t n_ctx, float theta, float* out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 1 || B > kMaxAttnBatch || !attn_shape_ok(H, H_kv, D)) return FMLP_ERR_INVALID_ARG;
+  if (n_ctx < 1 || n_max < n_ctx || (int64_t)B * H_kv * n_max > (int64_t)INT32_MAX)
+    return FMLP_ERR_INVALID_ARG;
+  if (!(theta > 0.f) || !std::isfinite(theta)) return FMLP_ERR_INVALID_ARG;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !out || !workspace)
+    return FMLP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)pos & 3u))
+    return FMLP_ERR_INVALID_ARG;
+  if (workspace_bytes < attn_layout(B, H, H_kv, D).total) return FMLP_ERR_INVALID_ARG;
+  const DeviceInfo* dev = nullptr;
+  fmlp_status st = device_for_launch(&dev);
+  if (st != FMLP_OK) return st;
+  cudaError_t e = launch_attn_decode(q, k_new, v_new, k_cache, v_cache, pos, B, H, H_kv, D,
+                                     n_max, (int)n_ctx, theta, out, workspace, *dev,
+                                     (cudaStream_t)stream);
+  return e == cudaSuccess ? FMLP_OK : cuda_fail(e);
+}
+
 fmlp_status fmlp_device_status(void* workspace, void* stream) {
   if (!workspace || !aligned16(workspace)) return FMLP_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
@@ -433,7 +462,8 @@ fmlp_status fmlp_device_status(void* workspace, void* stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
-  return word & kStatusTimeout ? FMLP_ERR_TIMEOUT : FMLP_OK;
+  if (word & kStatusTimeout) return FMLP_ERR_TIMEOUT;
+  return word & kStatusBadInput ? FMLP_ERR_INVALID_ARG : FMLP_OK;
 }
 
 }  // extern "C"

@@ -45,6 +45,7 @@ constexpr int kFusedMaxM = 4;  // token rows handled by the fused decode kernel
 WorkspaceLayout workspace_layout(int64_t M, int64_t d, int64_t I);
 
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBadInput = 2u;  // a device-side input out of range (attention position)
 
 // Count of kernels enqueued by the library (fmlp_kernel_launch_count).
 void note_launches(int n);
@@ -145,6 +146,20 @@ cudaError_t launch_forward_q8(const void* x, int64_t M, const void* gamma, float
                               const float* Wds, int64_t d, int64_t I, const void* residual,
                               float* out, void* out_bf16, void* a, uint32_t* status,
                               const DeviceInfo& dev, cudaStream_t stream);
+
+// Token-phase attention (csrc/attn.cu): GKVC append + TPSFLAT-style fused
+// RoPE / QK^T / softmax / PV over the cache.
+struct AttnLayout {
+  size_t counters = 0;  // [B H_kv] uint32 arrival counters (zero between calls)
+  size_t partials = 0;  // f32 pieces of the segments split over CTAs
+  size_t total = 0;
+};
+bool attn_shape_ok(int H, int H_kv, int D);
+AttnLayout attn_layout(int64_t B, int H, int H_kv, int D);
+cudaError_t launch_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                               void* v_cache, const int32_t* pos, int64_t B, int H, int H_kv,
+                               int D, int64_t n_max, int n_ctx, float theta, float* out,
+                               void* workspace, const DeviceInfo& dev, cudaStream_t stream);
 
 // out = residual or zero (for a down GEMM with no gate-up prologue before it).
 cudaError_t launch_out_init(float* out, const void* residual, int64_t M, int64_t d,

@@ -45,21 +45,29 @@ cudaError_t encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t row
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t encode_tmap_kblocks_bf16(CUtensorMap* map, const void* base, uint64_t rows,
-                                     uint64_t cols, uint64_t row_bytes, uint32_t box_rows,
-                                     uint32_t box_kblocks) {
+cudaError_t encode_tmap_blocks_bf16(CUtensorMap* map, const void* base, uint64_t rows,
+                                    uint64_t cols, uint64_t row_bytes, uint32_t block_cols,
+                                    uint32_t box_rows, uint32_t box_blocks,
+                                    CUtensorMapSwizzle swizzle) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   cudaError_t e = encoder(&fn);
   if (e != cudaSuccess) return e;
-  if (cols % 64 != 0) return cudaErrorInvalidValue;
-  const cuuint64_t dims[3] = {64, rows, cols / 64};
-  const cuuint64_t strides[2] = {row_bytes, 128};
-  const cuuint32_t box[3] = {64, box_rows, box_kblocks};
+  if (block_cols == 0 || cols % block_cols != 0) return cudaErrorInvalidValue;
+  const cuuint64_t dims[3] = {block_cols, rows, cols / block_cols};
+  const cuuint64_t strides[2] = {row_bytes, (cuuint64_t)block_cols * 2};
+  const cuuint32_t box[3] = {block_cols, box_rows, box_blocks};
   const cuuint32_t elem[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t encode_tmap_kblocks_bf16(CUtensorMap* map, const void* base, uint64_t rows,
+                                     uint64_t cols, uint64_t row_bytes, uint32_t box_rows,
+                                     uint32_t box_kblocks) {
+  return encode_tmap_blocks_bf16(map, base, rows, cols, row_bytes, 64, box_rows, box_kblocks,
+                                 CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace fmlp

@@ -24,4 +24,13 @@ cudaError_t encode_tmap_kblocks_bf16(CUtensorMap* map, const void* base, uint64_
                                      uint64_t cols, uint64_t row_bytes, uint32_t box_rows,
                                      uint32_t box_kblocks);
 
+// The same view with blocks of block_cols columns (32 with the 64-byte
+// swizzle, 64 with the 128-byte one): a box of box_rows x block_cols x
+// box_blocks lands as box_blocks consecutive box_rows x (2 block_cols)-byte
+// tiles.
+cudaError_t encode_tmap_blocks_bf16(CUtensorMap* map, const void* base, uint64_t rows,
+                                    uint64_t cols, uint64_t row_bytes, uint32_t block_cols,
+                                    uint32_t box_rows, uint32_t box_blocks,
+                                    CUtensorMapSwizzle swizzle);
+
 }  // namespace fmlp
