@@ -42,6 +42,8 @@ TILE_T = 16
 METRIC = "fused-MLP weight-stream GB/s (% B200 HBM peak) and tokens/s per layer at 1 GPU"
 # decode workloads also measured on this library's int8 weights (entries "<name>_q8")
 Q8_WORKLOADS = ["phi3_decode", "llama8b_decode_m1"]
+# the token-phase attention step on the same models' attention shapes
+ATTN_BENCH = ["phi3_attn", "llama8b_attn"]
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
@@ -81,6 +83,7 @@ def measured_peaks() -> dict:
 KERNEL_SOURCES = {
     "fused_decode": ["stream.cu", "ring.cuh", "common.cuh", "internal.h"],
     "q8_stream": ["q8.cu", "ring.cuh", "common.cuh", "internal.h"],
+    "attn_decode": ["attn.cu", "ring.cuh", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
     "tc_gemm": ["tc.cu", "tcgen05.cuh", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
     "tc_layer": ["layer.cu", "tcgen05.cuh", "common.cuh", "internal.h", "tmap.cu", "tmap.h"],
 }
@@ -647,6 +650,168 @@ def measure_sub_workload(fm, w: wl.Workload, dev, args, barrier, max_over_ranks,
     return entry
 
 
+def attn_bytes(w: wl.AttnWorkload) -> int:
+    """Algorithmic bytes of one attention step of one layer: the held K and V
+    rows read, the new rows written, q / k / v / positions read and out written."""
+    B, H, Hk, D = w.B, w.H, w.H_kv, w.D
+    return (2 * B * Hk * (w.n_ctx - 1) * D * 2 + B * H * D * 2 + 2 * B * Hk * D * 2 + 4 * B
+            + 2 * B * Hk * D * 2 + B * H * D * 4)
+
+
+class AttnRun:
+    """One attention workload resident on the GPU: every layer's K and V cache
+    regions, the new token's q / k / v and positions, one output per layer;
+    step() runs fmlp_attn_decode once per layer."""
+
+    def __init__(self, fm, w: wl.AttnWorkload, dev, seed0: int):
+        self.fm, self.w, self.dev, self.L = fm, w, dev, w.layers
+        p0 = wl.make_attn_problem(w.B, w.H, w.H_kv, w.D, w.n_max, seed=seed0)
+        self.host = p0                                  # layer 0's inputs, for the oracle
+        self.q, self.k_new, self.v_new = (p0[k].to(dev) for k in ("q", "k_new", "v_new"))
+        self.pos_host = torch.full((w.B,), w.n_ctx - 1, dtype=torch.int32)
+        self.pos = self.pos_host.to(dev)
+        self.caches = [(p0["k_cache"].to(dev), p0["v_cache"].to(dev))]
+        for l in range(1, self.L):
+            pl = wl.make_attn_problem(w.B, w.H, w.H_kv, w.D, w.n_max, seed=seed0 + l)
+            self.caches.append((pl["k_cache"].to(dev), pl["v_cache"].to(dev)))
+        self.outs = torch.empty(self.L, w.B, w.H, w.D, dtype=torch.float32, device=dev)
+        self.ws = torch.zeros(fm.fmlp_attn_workspace_bytes(w.B, w.H, w.H_kv, w.D),
+                              dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.graph, self.per_step, self.outs_last = None, None, None
+
+    def step(self, ins=None, outs=None, stream=None):
+        q, k, v, pos = ins if ins is not None else (self.q, self.k_new, self.v_new, self.pos)
+        outs = self.outs if outs is None else outs
+        for l, (kc, vc) in enumerate(self.caches):
+            self.fm.fmlp_attn_decode(q, k, v, kc, vc, pos, self.w.n_ctx, self.w.theta, outs[l],
+                                     self.ws, stream=stream)
+
+    capture = WorkloadRun.capture
+    run_steps = WorkloadRun.run_steps
+    timed = WorkloadRun.timed
+    step_estimate_ms = WorkloadRun.step_estimate_ms
+
+    def e2e(self, steps: int, barrier, max_over_ranks) -> tuple:
+        """As WorkloadRun.e2e: every step copies q, k, v and the positions in
+        from pinned host memory and every layer's out back, double-buffered on
+        copy streams.  Returns (ms, h2d bytes, d2h bytes)."""
+        stream = self.stream
+        host_in = [t.pin_memory() for t in (self.host["q"], self.host["k_new"], self.host["v_new"],
+                                            self.pos_host)]
+        dev_in = [[torch.empty_like(t, device=self.dev) for t in host_in] for _ in range(2)]
+        outs_host = [torch.empty(self.outs.shape, dtype=torch.float32).pin_memory()
+                     for _ in range(2)]
+        outs_dev = [self.outs, torch.empty_like(self.outs)]
+        copy_in, copy_out = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_step(i):
+            b = i & 1
+            copy_in.wait_event(ev_done[b])
+            with torch.cuda.stream(copy_in):
+                for d, h in zip(dev_in[b], host_in):
+                    d.copy_(h, non_blocking=True)
+            ev_in[b].record(copy_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])
+            self.step(ins=dev_in[b], outs=outs_dev[b], stream=stream)
+            ev_done[b].record(stream)
+            copy_out.wait_event(ev_done[b])
+            with torch.cuda.stream(copy_out):
+                outs_host[b].copy_(outs_dev[b], non_blocking=True)
+            ev_out[b].record(copy_out)
+
+        e2e_step(0)
+        e2e_step(1)
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        copy_in.wait_stream(stream)
+        for i in range(steps):
+            e2e_step(i)
+        stream.wait_event(ev_out[0])
+        stream.wait_event(ev_out[1])
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        self.outs_last = outs_dev[(steps - 1) & 1]
+        return (max_over_ranks(f0.elapsed_time(f1)),
+                sum(t.numel() * t.element_size() for t in host_in),
+                outs_host[0].numel() * outs_host[0].element_size())
+
+    def release(self) -> None:
+        self.graph = None
+        self.caches = []
+        self.outs = self.outs_last = None
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def attn_oracle_check(run: AttnRun, outs) -> dict:
+    """Layer 0's output of the last end-to-end pass against the oracle's step on
+    the same inputs (every sequence and head)."""
+    import oracle
+    dec = lambda t: oracle.decode_bf16(wl.bf16_bits(t))  # noqa: E731
+    h = run.host
+    ref, _, _ = oracle.token_attention(dec(h["q"]), dec(h["k_new"]), dec(h["v_new"]),
+                                       dec(h["k_cache"]), dec(h["v_cache"]),
+                                       run.pos_host.numpy(), run.w.theta)
+    got = outs[0].cpu().double().numpy()
+    norm = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    elem = float(np.max(np.abs(got - ref)) / np.max(np.abs(ref)))
+    return {"layer": 0, "normwise": float(f"{norm:.3e}"), "per_element": float(f"{elem:.3e}"),
+            "within_bar": bool(norm <= 1e-4 and elem <= 1e-3), "bar": "normwise 1e-4, per element 1e-3"}
+
+
+def measure_attn_workload(fm, w: wl.AttnWorkload, dev, args, barrier, max_over_ranks, rank: int,
+                          world: int) -> dict:
+    """A `workloads` entry for the token-phase attention step: timed for at
+    least --min-seconds, one fmlp_attn_decode per layer back to back in a CUDA
+    graph (one kernel per layer), with its roofline, end-to-end pass, oracle
+    check and clocks."""
+    run = AttnRun(fm, w, dev, seed0=1000 * rank)
+    run.capture(args.warmup, use_graph=not args.no_graph)
+    est = run.step_estimate_ms()
+    steps = max(args.steps, int(np.ceil(args.min_seconds * 1e3 / max(est, 1e-3))))
+    ms, launches, clocks = run.timed(steps, barrier, max_over_ranks)
+    ms_step = ms / steps
+    e2e_steps = max(2, min(4000, int(np.ceil(0.5e3 / max(est, 1e-3)))))
+    e2e_ms, h2d, d2h = run.e2e(e2e_steps, barrier, max_over_ranks)
+    bytes_step = run.L * attn_bytes(w)
+    (peak, src), _ = peaks_of(sustained=True)
+    gbs = job_gbs(bytes_step, steps, world, ms)
+    kms = ms_step / run.L
+    achieved = attn_bytes(w) / (kms / 1e3) / 1e9
+    entry = {
+        "config": {"B": w.B, "H": w.H, "H_kv": w.H_kv, "D": w.D, "n_ctx": w.n_ctx, "n_max": w.n_max,
+                   "rope_theta": w.theta, "layers": run.L,
+                   "kv_cache_per_gpu_GB": round(2 * w.B * w.H_kv * w.n_max * w.D * 2 * run.L / 1e9, 3)},
+        "value": round(gbs, 2), "unit": "GB/s", "hbm_frac": round(gbs / world / peak, 4),
+        "tokens_per_s_per_layer": round(w.B * run.L * steps * world / (ms / 1e3), 1),
+        "ms_per_layer": round(kms, 5), "steps": steps, "timed_ms": round(ms, 2),
+        "roofline": {"bound": "hbm", "kernel": "attn_decode", "achieved": round(achieved, 2),
+                     "peak": peak, "peak_source": src, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": recorded_traffic("attn_decode", w.name),
+                     "algorithmic_per_launch": attn_bytes(w), "avg_launch_ms": round(kms, 5),
+                     "launch_timing": "timed region / launches (one kernel per layer, back to back "
+                                      "in a CUDA graph)"},
+        "e2e": {"value": round(job_gbs(bytes_step, e2e_steps, world, e2e_ms), 2), "unit": "GB/s",
+                "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches, "cuda_graph": run.graph is not None,
+        "device_status": fm.fmlp_status_string(fm.fmlp_device_status(run.ws)),
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_oracle_check:
+        entry["check_vs_oracle"] = attn_oracle_check(run, run.outs_last)
+    run.release()
+    return entry
+
+
 def run_ours(args) -> None:
     rank, world, local = dist_env()
     if world > 1:
@@ -703,9 +868,13 @@ def run_ours(args) -> None:
     # entry each
     subs = {}
     names = [] if args.workloads == "none" else (
-        list(wl.WORKLOADS) + [n + "_q8" for n in Q8_WORKLOADS] if args.workloads == "all"
-        else args.workloads.split(","))
+        list(wl.WORKLOADS) + [n + "_q8" for n in Q8_WORKLOADS] + ATTN_BENCH
+        if args.workloads == "all" else args.workloads.split(","))
     for name in names:
+        if name in wl.ATTN_WORKLOADS:
+            subs[name] = measure_attn_workload(fm, wl.ATTN_WORKLOADS[name], dev, args, barrier,
+                                               max_over_ranks, rank, world)
+            continue
         quant = name.endswith("_q8")
         subs[name] = measure_sub_workload(fm, wl.WORKLOADS[name[:-3] if quant else name], dev,
                                           args, barrier, max_over_ranks, rank, world, quant=quant)
