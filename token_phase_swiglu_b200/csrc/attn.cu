@@ -52,6 +52,40 @@ constexpr int kAttnConsumerThreads = kAttnWarps * 32;
 constexpr int kAttnBar = 1;                                     // consumer-only named barrier
 constexpr int kAttnMaxCtas = 256;
 constexpr int kAttnTileBytesPerBlock = kAttnRows * 64;          // 64 rows x 32 bf16
+// Head dimensions that are multiples of 64 are copied in 64-column blocks with
+// the 128-byte swizzle (128-byte pieces per row), the others (96) in
+// 32-column blocks with the 64-byte swizzle.
+constexpr bool kAttnWideBlocks = true;
+// Consumer warps waiting for their next stage sleep between polls instead of
+// taking issue slots from the warps that are computing.
+constexpr bool kAttnBackoff = true;
+
+template <int DC>
+struct AttnTile {
+  static constexpr bool wide = kAttnWideBlocks && DC % 2 == 0;
+  static constexpr int block_cols = wide ? 64 : 32;
+  static constexpr int row_bytes = block_cols * 2;           // of one block
+  static constexpr int block_bytes = kAttnRows * row_bytes;
+  // byte offset of element (row, column d) in a tile
+  __device__ static __forceinline__ int offset(int row, int d) {
+    const int zb = d / block_cols, col = d % block_cols;
+    const int sw = wide ? (row & 7) : ((row >> 1) & 3);
+    return zb * block_bytes + row * row_bytes + ((((col >> 3) ^ sw)) << 4) + (col & 7) * 2;
+  }
+};
+
+__device__ __forceinline__ bool attn_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                          volatile int* abort) {
+  if (!kAttnBackoff) return mbar_wait_bounded(bar, parity, limit_ns, abort);
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (mbar_test(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
 
 struct AttnParams {
   CUtensorMap k_map;        // cache as [B H_kv N_max rows x D] bf16: 32-column blocks, 64-B swizzle
@@ -256,8 +290,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
         if (rows == 0) continue;
         if (k % kAttnGroups == grp) {
           const int slot = k % ring.stages;
-          if (!mbar_wait_bounded(&ring.full[slot], (uint32_t)((k / ring.stages) & 1), p.ctl.wait_ns,
-                                 &st.abort)) {
+          if (!attn_wait(&ring.full[slot], (uint32_t)((k / ring.stages) & 1), p.ctl.wait_ns,
+                         &st.abort)) {
             if (lane == 0) flag_timeout(&st, p.ctl.status);
             ok = false;
             break;
@@ -270,12 +304,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
           uint64_t sacc[G];
 #pragma unroll
           for (int h = 0; h < G; ++h) sacc[h] = 0ull;
-          const int rsw = (r >> 1) & 3;  // the 64-byte swizzle of row r
 #pragma unroll
           for (int z = 0; z < DC; ++z) {
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-              const uint4 kv = lds128(kt + z * kAttnTileBytesPerBlock + r * 64 + ((cc ^ rsw) << 4));
+              const uint4 kv = lds128(kt + AttnTile<DC>::offset(r, z * 32 + cc * 8));
               const uint64_t k0 = bf16x2_f32x2(kv.x), k1 = bf16x2_f32x2(kv.y);
               const uint64_t k2 = bf16x2_f32x2(kv.z), k3 = bf16x2_f32x2(kv.w);
 #pragma unroll
@@ -309,7 +342,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
           __syncwarp();
           // PV: lane owns dimensions lane + 32 i
           const int nr = min(max(rows - half * 32, 0), 32);
-          const int lsw = lane >> 3, lo = (lane & 7) * 2;
           int rr = 0;
           for (; rr + 4 <= nr; rr += 4) {
             float4 pp[G];
@@ -318,11 +350,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               const int row = half * 32 + rr + q4;
-              const uint8_t* vr = vt + row * 64 + ((lsw ^ ((row >> 1) & 3)) << 4) + lo;
               float v[DC];
 #pragma unroll
               for (int i = 0; i < DC; ++i)
-                v[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vr + i * kAttnTileBytesPerBlock));
+                v[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                    vt + AttnTile<DC>::offset(row, lane + 32 * i)));
 #pragma unroll
               for (int h = 0; h < G; ++h) {
                 const float ph = q4 == 0 ? pp[h].x : q4 == 1 ? pp[h].y : q4 == 2 ? pp[h].z : pp[h].w;
@@ -333,10 +365,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
           }
           for (; rr < nr; ++rr) {
             const int row = half * 32 + rr;
-            const uint8_t* vr = vt + row * 64 + ((lsw ^ ((row >> 1) & 3)) << 4) + lo;
 #pragma unroll
             for (int i = 0; i < DC; ++i) {
-              const float v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vr + i * kAttnTileBytesPerBlock));
+              const float v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                  vt + AttnTile<DC>::offset(row, lane + 32 * i)));
 #pragma unroll
               for (int h = 0; h < G; ++h) acc[h][i] = fmaf(pw[h * 32 + rr], v, acc[h][i]);
             }
@@ -402,17 +434,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
           __threadfence();
           for (int t = ct; t < G * D; t += kAttnConsumerThreads) {
             const int h = t / D, d = t % D;
+            // the pieces' loads are independent: unrolled so that they overlap
+            // (an L2 round trip each otherwise); an empty piece has m = -inf,
+            // weight exp2(-inf) = 0 and zero sums
             float M = -CUDART_INF_F;
+#pragma unroll 4
             for (int cc = cf; cc <= cl; ++cc)
               M = fmaxf(M, __ldcg(p.partials + (size_t)(cc + s) * G * (2 + D) + h * (2 + D)));
             float A = 0.f, L = 0.f;
+#pragma unroll 4
             for (int cc = cf; cc <= cl; ++cc) {
               const float* pc = p.partials + (size_t)(cc + s) * G * (2 + D) + h * (2 + D);
-              const float mc = __ldcg(pc);
-              if (mc == -CUDART_INF_F) continue;
+              const float mc = __ldcg(pc), lc = __ldcg(pc + 1), ac = __ldcg(pc + 2 + d);
               const float f = exp2f(mc - M);
-              A = fmaf(f, __ldcg(pc + 2 + d), A);
-              L = fmaf(f, __ldcg(pc + 1), L);
+              A = fmaf(f, ac, A);
+              L = fmaf(f, lc, L);
             }
             p.out[((int64_t)b * p.H + (int64_t)g * G + h) * D + d] = A / L;
           }
@@ -478,11 +514,14 @@ cudaError_t launch_attn_t(AttnParams& p, const DeviceInfo& dev, cudaStream_t str
   p.stages = pl.stages;
   p.stage_bytes = pl.stage_bytes;
   const uint64_t rows = (uint64_t)p.B * p.H_kv * (uint64_t)p.n_max;
-  e = encode_tmap_blocks_bf16(&p.k_map, p.k_cache, rows, (uint64_t)p.D, (uint64_t)p.D * 2, 32,
-                              kAttnRows, DC, CU_TENSOR_MAP_SWIZZLE_64B);
+  using Tile = AttnTile<DC>;
+  const CUtensorMapSwizzle sw = Tile::wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const uint32_t blocks = (uint32_t)(p.D / Tile::block_cols);
+  e = encode_tmap_blocks_bf16(&p.k_map, p.k_cache, rows, (uint64_t)p.D, (uint64_t)p.D * 2,
+                              Tile::block_cols, kAttnRows, blocks, sw);
   if (e == cudaSuccess)
-    e = encode_tmap_blocks_bf16(&p.v_map, p.v_cache, rows, (uint64_t)p.D, (uint64_t)p.D * 2, 32,
-                                kAttnRows, DC, CU_TENSOR_MAP_SWIZZLE_64B);
+    e = encode_tmap_blocks_bf16(&p.v_map, p.v_cache, rows, (uint64_t)p.D, (uint64_t)p.D * 2,
+                                Tile::block_cols, kAttnRows, blocks, sw);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)pl.ctas);
