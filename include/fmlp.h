@@ -287,14 +287,15 @@ FMLP_API size_t fmlp_attn_workspace_bytes(int64_t B, int H, int H_kv, int D);
  *              (N_p + N_r of Eq(2)); rows 0..pos[b]-1 hold the earlier tokens.
  *              The call writes row pos[b] of every KV head of sequence b --
  *              the rotated key rounded to bf16 (nearest even), and v_new --
- *              at the Eq(2) offset ((b H_kv + g) n_max + pos[b]) D, and reads
- *              nothing past it.
+ *              at the Eq(2) offset ((b H_kv + g) n_max + pos[b]) D; rows past
+ *              pos[b] do not enter the result.
  *   pos      : int32 [B] on the device, the new token's position (rows held);
  *              0 <= pos[b] < n_ctx <= n_max.  A position outside that range is
  *              not processed: its sequence's outputs and cache are left as
  *              they were and fmlp_device_status reports FMLP_ERR_INVALID_ARG.
- *   n_ctx    : host-side bound on every pos[b] + 1; the work is split over
- *              n_ctx rows per sequence, so a tight bound balances best.
+ *   n_ctx    : host-side bound on every pos[b] + 1.  The call streams the
+ *              rows below n_ctx of every region (rows at and past pos[b] are
+ *              read and not used), so n_ctx should be tight: max(pos) + 1.
  *   theta    : RoPE base (> 0): angle_i = pos * theta^(-2i/D), pairs (i, i + D/2)
  *   out      : f32 [B x H x D]: o_h = softmax(q'_h . K_g / sqrt(D)) V_g with
  *              g = h / (H / H_kv), accumulated in f32

@@ -105,8 +105,8 @@ struct AttnParams {
   int n_ctx;                // every position < n_ctx
   int useg;                 // units per segment: ceil(n_ctx / 64)
   int64_t units;            // segments x useg
-  float theta;
   float qscale;             // log2(e) / sqrt(D)
+  double inv_freq[64];      // theta^(-2i/D), i < D/2 (binary64, from the host)
   int stages, stage_bytes;
 };
 
@@ -180,24 +180,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
   if (warp == 0) {
     // ---------------- producer ----------------
     if (lane == 0) {
-      int total = 0;  // stages this CTA will issue
-      for (int64_t s = seg0; s <= seg1; ++s) {
-        const int pb = __ldg(p.pos + s / p.H_kv);
-        if (bad_position(pb, p.n_ctx)) continue;
-        const int64_t a = max(u0, s * p.useg) - s * p.useg, e = min(u1, (s + 1) * p.useg) - s * p.useg;
-        const int64_t live = (pb + kAttnRows - 1) / kAttnRows;  // units holding rows < pb
-        const int64_t n = (e < live ? e : live) - a;
-        total += n > 0 ? (int)n : 0;
-      }
+      // every unit of the range, whatever the positions (the consumers mask the
+      // rows at and past a sequence's position), so the first copies need no
+      // read of the positions
+      const int total = (int)(u1 - u0);
       Producer pr{ring, &st, p.ctl, evict_first_policy(), total};
       const uint32_t tile = (uint32_t)(DC * kAttnTileBytesPerBlock);
       bool ok = true;
       for (int64_t s = seg0; s <= seg1 && ok; ++s) {
-        const int pb = __ldg(p.pos + s / p.H_kv);
-        if (bad_position(pb, p.n_ctx)) continue;
         for (int64_t u = max(u0, s * p.useg); u < min(u1, (s + 1) * p.useg); ++u) {
           const int j = (int)(u - s * p.useg);
-          if (unit_rows(j, pb) == 0) continue;
           if (!pr.acquire()) {
             ok = false;
             break;
@@ -226,6 +218,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
       const int pb = __ldg(p.pos + b);
       if (bad_position(pb, p.n_ctx)) {
         if (ct == 0) atomicOr(p.ctl.status, kStatusBadInput);
+        // its stages arrive all the same: take them and give them back
+        for (int64_t u = max(u0, s * p.useg); u < min(u1, (s + 1) * p.useg) && ok; ++u, ++k) {
+          if (k % kAttnGroups != grp) continue;
+          const int slot = k % ring.stages;
+          if (!attn_wait(&ring.full[slot], (uint32_t)((k / ring.stages) & 1), p.ctl.wait_ns,
+                         &st.abort)) {
+            if (lane == 0) flag_timeout(&st, p.ctl.status);
+            ok = false;
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ring.empty[slot]);
+        }
+        if (consumer_barrier_any<kAttnConsumerThreads>(kAttnBar, !ok)) break;
         continue;
       }
       const int64_t sa = max(u0, s * p.useg), se = min(u1, (s + 1) * p.useg);
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
       // RoPE at position pb: angles in binary64, then the rotated q (and, in
       // the owner, the new k and v, which it also appends to the cache).
       for (int i = ct; i < D / 2; i += kAttnConsumerThreads) {
-        const double a = (double)pb * pow((double)p.theta, -2.0 * i / D);
+        const double a = (double)pb * p.inv_freq[i];
         double sd, cd;
         sincos(a, &sd, &cd);
         sh.cs[i] = (float)cd;
@@ -286,8 +292,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_decode(const __grid_cons
         for (int i = 0; i < DC; ++i) acc[h][i] = 0.f;
       }
       for (int64_t u = sa; u < se && ok; ++u) {
-        const int rows = unit_rows((int)(u - s * p.useg), pb);
-        if (rows == 0) continue;
+        const int rows = unit_rows((int)(u - s * p.useg), pb);  // 0 past the position
         if (k % kAttnGroups == grp) {
           const int slot = k % ring.stages;
           if (!attn_wait(&ring.full[slot], (uint32_t)((k / ring.stages) & 1), p.ctl.wait_ns,
@@ -592,7 +597,7 @@ cudaError_t launch_attn_decode(const void* q, const void* k_new, const void* v_n
   p.G = H / H_kv;
   p.n_max = n_max;
   p.n_ctx = n_ctx;
-  p.theta = theta;
+  for (int i = 0; i < D / 2; ++i) p.inv_freq[i] = std::pow((double)theta, -2.0 * i / D);
   p.qscale = (float)(1.4426950408889634 / std::sqrt((double)D));  // log2(e) / sqrt(D)
   switch (D) {
     case 64: return launch_attn_g<2>(p, dev, stream);
