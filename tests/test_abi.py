@@ -163,3 +163,48 @@ def test_binding_checks_shapes_and_device_before_the_library():
         fm.fmlp_down_proj(bf(M, I), Wd, out[:, :8], ws)
     with pytest.raises(ValueError, match="shape"):
         fm.fmlp_gate_up_swiglu(x, gamma, 1e-5, packed, 16, bf(M + 1, I), ws)
+
+
+def test_attention_workspace_and_rejections():
+    """fmlp_attn_workspace_bytes / fmlp_attn_decode on the host: the shapes the
+    kernel takes, the workspace it needs, and every argument it refuses before
+    any CUDA call."""
+    L = fm.lib
+    # counters (one per sequence x KV head) + one f32 piece (m, l, acc[D]) per head per slot
+    n = L.fmlp_attn_workspace_bytes(8, 32, 8, 128)
+    assert n >= 256 + 8 * 8 * 4 + (148 + 64) * 4 * (2 + 128) * 4
+    assert L.fmlp_attn_workspace_bytes(1, 32, 32, 96) > 0
+    for B, H, H_kv, D in [(1, 32, 32, 80), (1, 12, 8, 64), (1, 48, 3, 64), (0, 8, 8, 64),
+                          (1, 8, 8, 256), (1, 0, 1, 64)]:
+        assert L.fmlp_attn_workspace_bytes(B, H, H_kv, D) == 0, (B, H, H_kv, D)
+    W = 0x40000
+    good = dict(q=A, k=A, v=A, kc=A, vc=A, pos=A, B=2, H=8, H_kv=2, D=64, n_max=256, n_ctx=200,
+                theta=10000.0, out=A, ws=W, wsb=1 << 20)
+    bad = [dict(D=80), dict(H=9), dict(n_ctx=300), dict(n_ctx=0), dict(theta=0.0),
+           dict(theta=float("inf")), dict(q=None), dict(pos=A + 2), dict(out=MIS), dict(kc=MIS),
+           dict(wsb=16), dict(B=0), dict(n_max=1 << 30, B=8, H=8, H_kv=8)]
+    for kw in bad:
+        a = good | kw
+        st = L.fmlp_attn_decode(a["q"], a["k"], a["v"], a["kc"], a["vc"], a["pos"], a["B"], a["H"],
+                                a["H_kv"], a["D"], a["n_max"], a["n_ctx"], a["theta"], a["out"],
+                                a["ws"], a["wsb"], None)
+        assert st == fm.FMLP_ERR_INVALID_ARG, kw
+
+
+def test_attention_binding_checks_before_the_library():
+    import torch
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    B, H, H_kv, D, n_max = 2, 4, 2, 64, 128
+    q, kn, vn = bf(B, H, D), bf(B, H_kv, D), bf(B, H_kv, D)
+    kc, vc = bf(B, H_kv, n_max, D), bf(B, H_kv, n_max, D)
+    pos = torch.zeros(B, dtype=torch.int32)
+    out = torch.zeros(B, H, D)
+    ws = torch.zeros(fm.fmlp_attn_workspace_bytes(B, H, H_kv, D), dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        fm.fmlp_attn_decode(q, kn, vn, kc, vc, pos.to(torch.int64), n_max, 1e4, out, ws)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_attn_decode(q, kn, vn, kc, bf(B, H_kv, n_max - 1, D), pos, n_max, 1e4, out, ws)
+    with pytest.raises(ValueError, match="shape"):
+        fm.fmlp_attn_decode(q, bf(B, H, D), vn, kc, vc, pos, n_max, 1e4, out, ws)
+    with pytest.raises(ValueError, match="CUDA"):
+        fm.fmlp_attn_decode(q, kn, vn, kc, vc, pos, n_max, 1e4, out, ws)
