@@ -593,7 +593,8 @@ def oracle_check(run: WorkloadRun, got_outs) -> dict:
     rows = check_rows(w.M)
     b = layer_bits(w, run.seed0, 0)
     import oracle
-    if run.quant:   # the block on the dequantized int8 weights
+    t0 = time.perf_counter()
+    if run.quant:   # the block on the dequantized int8 weights (quantization included)
         dec = oracle.decode_bf16
         qs = [oracle.quantize_rows(dec(b[k])) for k in ("W_gate", "W_up", "W_down")]
         ref = oracle.fused_mlp_q8(dec(b["x"][rows]), dec(b["gamma"]), EPS, *qs[0], *qs[1],
@@ -601,9 +602,15 @@ def oracle_check(run: WorkloadRun, got_outs) -> dict:
     else:
         ref = oracle.fused_mlp_bf16(b["x"][rows], b["gamma"], EPS, b["W_gate"], b["W_up"],
                                     b["W_down"])
+    dt = time.perf_counter() - t0
     got = got_outs[0].cpu().double().numpy()[rows]
     norm = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
     elem = float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-300))
+    nbytes = (q8_bytes if run.quant else algorithmic_bytes)(len(rows), w.d, w.I)
+    run.cpu_baseline = {
+        "value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+        "host_cores": host_cores(), "kind": "oracle",
+        "sample": f"this check: layer 0, {len(rows)} token row(s), through the fp64 oracle, {dt:.2f} s"}
     return {"layer": 0, "rows": len(rows), "normwise": float(f"{norm:.3e}"),
             "per_element": float(f"{elem:.3e}"), "within_bar": bool(norm <= 2e-3 and elem <= 1e-2)}
 
@@ -646,6 +653,7 @@ def measure_sub_workload(fm, w: wl.Workload, dev, args, barrier, max_over_ranks,
     }
     if rank == 0 and not args.no_oracle_check:
         entry["check_vs_oracle"] = oracle_check(run, run.outs_last)
+        entry["cpu_baseline"] = run.cpu_baseline
     run.release()
     return entry
 
@@ -757,9 +765,15 @@ def attn_oracle_check(run: AttnRun, outs) -> dict:
     import oracle
     dec = lambda t: oracle.decode_bf16(wl.bf16_bits(t))  # noqa: E731
     h = run.host
-    ref, _, _ = oracle.token_attention(dec(h["q"]), dec(h["k_new"]), dec(h["v_new"]),
-                                       dec(h["k_cache"]), dec(h["v_cache"]),
-                                       run.pos_host.numpy(), run.w.theta)
+    args = (dec(h["q"]), dec(h["k_new"]), dec(h["v_new"]), dec(h["k_cache"]), dec(h["v_cache"]),
+            run.pos_host.numpy(), run.w.theta)
+    t0 = time.perf_counter()
+    ref, _, _ = oracle.token_attention(*args)
+    dt = time.perf_counter() - t0
+    run.cpu_baseline = {
+        "value": round(attn_bytes(run.w) / dt / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+        "host_cores": host_cores(), "kind": "oracle",
+        "sample": f"this check: layer 0's whole step through the fp64 oracle, {dt:.2f} s"}
     got = outs[0].cpu().double().numpy()
     norm = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
     elem = float(np.max(np.abs(got - ref)) / np.max(np.abs(ref)))
@@ -808,6 +822,7 @@ def measure_attn_workload(fm, w: wl.AttnWorkload, dev, args, barrier, max_over_r
     }
     if rank == 0 and not args.no_oracle_check:
         entry["check_vs_oracle"] = attn_oracle_check(run, run.outs_last)
+        entry["cpu_baseline"] = run.cpu_baseline
     run.release()
     return entry
 
