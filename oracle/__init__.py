@@ -22,7 +22,7 @@ llama.cpp PR #29948 paragraph on interleaved gate/up rows):
 
 and the gate/up interleave, a pure permutation of rows at tile granularity.
 
-``quant.py`` restates this build's int8 weight format (the pages name
+``quant.py`` restates the library's own int8 weight format (the pages name
 quantized weight streaming but give no format) and the block on it.
 
 ``attn.py`` restates the token-phase attention step of the same pages

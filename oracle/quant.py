@@ -3,7 +3,7 @@
 The pages name quantized weight streaming over interleaved gate/up rows (the
 llama.cpp PR #29948 paragraph of "CUDAカーネル融合で推論が最大10%高速化",
 blog.cecily.jp: MMQ with the fused gate/up + GLU, Q4_K_M) but define no
-block format.  This build's own format, restated here plainly:
+block format.  The library's own format, restated here plainly:
 
   * a weight matrix W [rows x K] (K: the contraction axis -- d for the packed
     gate/up rows, I for W_down) is cut along K into groups of G = 64

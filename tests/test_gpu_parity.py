@@ -1,6 +1,6 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle.
 
-Bars (from the method's accuracy statement for this build):
+Bars (the library's accuracy contract):
   * the MLP output: normwise relative error <= 2e-3 and per-element error
     <= 1e-2 * max|O_ref| against the binary64 oracle;
   * diagnostic, tighter: against the oracle with its intermediate rounded to
