@@ -304,7 +304,7 @@ FMLP_API size_t fmlp_attn_workspace_bytes(int64_t B, int H, int H_kv, int D);
  *              reported FMLP_ERR_TIMEOUT or FMLP_ERR_INVALID_ARG through
  *              fmlp_device_status, zero it again before reuse.
  * Shapes taken: D in {64, 96, 128}; H / H_kv in {1, 2, 4, 8}; B * H_kv * n_max
- * < 2^31.  All pointers 16-byte aligned (pos 4-byte).  Runs after the
+ * + 64 < 2^31.  All pointers 16-byte aligned (pos 4-byte).  Runs after the
  * previous work on `stream` (which may have written the cache or pos).
  * Returns FMLP_ERR_INVALID_ARG before launching anything if an argument is
  * outside these limits.

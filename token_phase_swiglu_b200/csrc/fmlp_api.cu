@@ -432,7 +432,8 @@ fmlp_status fmlp_attn_decode(const void* q, const void* k_new, const void* v_new
                              int64_t n_max, int64_t n_ctx, float theta, float* out,
                              void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 1 || B > kMaxAttnBatch || !attn_shape_ok(H, H_kv, D)) return FMLP_ERR_INVALID_ARG;
-  if (n_ctx < 1 || n_max < n_ctx || (int64_t)B * H_kv * n_max > (int64_t)INT32_MAX)
+  // TMA row coordinates (int32) run to the end of the last 64-row unit
+  if (n_ctx < 1 || n_max < n_ctx || (int64_t)B * H_kv * n_max + 64 > (int64_t)INT32_MAX)
     return FMLP_ERR_INVALID_ARG;
   if (!(theta > 0.f) || !std::isfinite(theta)) return FMLP_ERR_INVALID_ARG;
   if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !out || !workspace)
