@@ -217,9 +217,13 @@ FMLP_API fmlp_status fmlp_quantize_q8(const void* W, int64_t rows, int64_t K, vo
  * fmlp_forward_q8 -- the MLP block (steps a1-a6) on int8 weights from
  * fmlp_quantize_q8: fmlp_forward with W_gate, W_up and W_down replaced by
  * their dequantized values q * s.  Decode batches only: 1 <= M <= 4 token
- * rows, d and I multiples of 512, M*d*4 and M*I*4 bytes within shared
- * memory (about 200 KB); other requests return FMLP_ERR_UNSUPPORTED.  About
- * 1.06 bytes of weights per element are streamed instead of 2.
+ * rows, d and I multiples of 512, and the M rows' activations in f32
+ * (M*d*4 and M*I*4 bytes) plus a ring of at least three stages within a
+ * CTA's shared memory (with I = 14336: up to 3 rows); other requests return
+ * FMLP_ERR_UNSUPPORTED before anything is launched.  About 1.06 bytes of
+ * weights per element are streamed instead of 2.  Every device-side wait is
+ * bounded; a kernel that gives one up sets the workspace status word
+ * (fmlp_device_status reports FMLP_ERR_TIMEOUT).
  *
  *   packed_q, packed_scales : fmlp_pack's [2I x d] matrix quantized (int8,
  *                             f32 [2I x d/64]) with the same tile_T

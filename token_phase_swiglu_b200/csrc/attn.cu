@@ -17,8 +17,8 @@
 // cut into units of 64 rows and split evenly over one CTA per SM (stream-K:
 // a CTA's range may end inside one segment and start inside another).  Warp
 // 0's elected lane streams each unit's K and V tiles into a ring of shared-
-// memory stages with two 3-D TMA copies (blocks of 32 columns, 64-byte
-// swizzle, so that a lane reading its own row meets no bank conflict).  Eight
+// memory stages with two 3-D TMA copies (swizzled column blocks, so that
+// lanes reading their own rows meet no bank conflict; see AttnTile).  Eight
 // consumer warps take the stages two at a time, 32 rows each: QK^T with one
 // row per lane (the G query heads of the KV head at once, q held in shared
 // memory, packed f32x2 FMAs), an online softmax in base 2 (scores carry
@@ -51,7 +51,7 @@ constexpr int kAttnThreads = (kAttnWarps + 1) * 32;             // warp 0 produc
 constexpr int kAttnConsumerThreads = kAttnWarps * 32;
 constexpr int kAttnBar = 1;                                     // consumer-only named barrier
 constexpr int kAttnMaxCtas = 256;
-constexpr int kAttnTileBytesPerBlock = kAttnRows * 64;          // 64 rows x 32 bf16
+constexpr int kAttnTileBytesPerBlock = kAttnRows * 64;          // per 32 columns of a tile
 // Head dimensions that are multiples of 64 are copied in 64-column blocks with
 // the 128-byte swizzle (128-byte pieces per row), the others (96) in
 // 32-column blocks with the 64-byte swizzle.
