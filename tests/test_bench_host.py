@@ -56,3 +56,28 @@ def test_bench_oracle_check_rows_reach_every_token_tile():
     assert rows[0] == 0 and rows[-1] == 2047 and len(rows) <= 80
     assert {r // 128 for r in rows} == set(range(16))
     assert {r // 256 for r in rows} == set(range(8))
+
+
+def test_int8_and_attention_byte_models():
+    # int8 layer: codes 3dI + scales 3dI/16 (one f32 per 64) + x, gamma, a, out
+    assert bench.q8_bytes(1, 4096, 14336) == 187_203_584
+    assert bench.q8_bytes(1, 3072, 8192) == 80_240_640
+    # attention step: the held K and V rows (n_ctx - 1 of them) + q, k, v, positions, new rows, out
+    w = wl.ATTN_WORKLOADS["llama8b_attn"]
+    held = 2 * w.B * w.H_kv * (w.n_ctx - 1) * w.D * 2
+    assert bench.attn_bytes(w) == held + w.B * w.H * w.D * 2 + 4 * w.B * w.H_kv * w.D * 2 \
+        + 4 * w.B + w.B * w.H * w.D * 4
+    assert round(bench.attn_bytes(wl.ATTN_WORKLOADS["phi3_attn"]) / 1e6, 2) == 50.36
+    assert w.kv_bytes == 2 * w.B * w.H_kv * w.n_ctx * w.D * 2
+
+
+def test_default_run_covers_every_workload_family():
+    """`--workloads all` (the default) measures the bf16 workloads, the int8 ones
+    and the attention step; every kernel with a traffic record has its sources listed."""
+    names = list(wl.WORKLOADS) + [n + "_q8" for n in bench.Q8_WORKLOADS] + bench.ATTN_BENCH
+    assert {"phi3_decode_q8", "llama8b_decode_m1_q8", "phi3_attn", "llama8b_attn"} <= set(names)
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for kernel in rec:
+        assert kernel in bench.KERNEL_SOURCES
+        for name in bench.KERNEL_SOURCES[kernel]:
+            assert os.path.exists(os.path.join(ROOT, "token_phase_swiglu_b200", "csrc", name))
